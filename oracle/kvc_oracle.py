@@ -1,0 +1,307 @@
+"""Plain fp64 CPU oracle for observation-window KV-cache compression.
+
+TEST INFRASTRUCTURE.  Only the test-suite, the package smoke check and the
+bench's CPU-baseline leg may import this module.  The CUDA library never calls
+it and shares no code with it.
+
+What it computes, step by step, in float64 from the stored inputs (fp32 values
+or bf16 bit patterns, both widened exactly):
+
+1. ``window_probs`` -- for each sequence b, KV head h, query head g of the GQA
+   group of h and window row i (absolute position p = len_b - w + i): the
+   logits z_j = scale * q . k_j for the keys j <= p, and the softmax
+   pi_j = exp(z_j - max z) / sum exp(z - max z).  Observation-window scoring of
+   SnapKV ("Variantes de l'attention et compression du cache KV", section
+   "Compresser un cache existant"); FastKV's saliency from the attention of the
+   recent window (FastKV, section 2.A).  The causal rule -- row i of a q-row
+   segment appended after S cached tokens sees keys up to S + i -- is from the
+   same attention-variants page, section "Quand la reutilisation est-elle
+   exacte ?".
+2. ``raw_scores`` -- raw[h][j] = sum over the G heads and w rows of pi_j.
+3. ``pool_prefix`` -- 1-D max-pool of raw over the prefix [0, P), P = len - w.
+4. ``select_topk`` -- per KV head the B - w prefix positions with the largest
+   pooled score (ties: lower index first), ascending, then the w window
+   positions.  Original positions are kept, never renumbered (attention-variants
+   page, section "Quand la reutilisation est-elle exacte ?").
+5. ``gather_kv`` -- byte copy of the retained rows into a compact cache.
+6. ``gqa_decode`` -- textbook softmax attention of one query per head over the
+   retained rows of its KV head (GQA head sharing: attention-variants page,
+   section "MHA et GQA").
+7. ``tsp_select`` / ``tsp_gather`` -- FastKV token-selective propagation
+   (FastKV, section 2.A): scores summed over all heads, pooled, one token set
+   of k_tsp prefix positions plus the window, hidden rows copied.
+8. ``cache_bytes`` -- 2 * L * S * n_kv * d_h * b (attention-variants page,
+   section "MHA et GQA").
+
+Readings of points the pages leave open (each also listed in the design doc):
+* logit scale: passed explicitly, 1/sqrt(d_h) by default;
+* GQA mapping: query head qh uses KV head qh // G (contiguous groups);
+* softmax domain: the whole visible row, window keys included; only prefix
+  positions are pooled and selected;
+* order: sum over heads and rows first, then pool;
+* pool: stride 1, same length, neighbours outside [0, P) ignored;
+* the per-head budget B counts the window (B - w prefix positions);
+  the TSP count k_tsp does not (k_tsp + w rows);
+* B >= len keeps every position; B < w is rejected; even pool sizes rejected.
+
+Parity pins for every function live in tests/test_oracle_pins.py; none of them
+re-types these formulas.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+# ----------------------------------------------------------------------------
+# inputs
+# ----------------------------------------------------------------------------
+def to_f64(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Stored representation -> float64 (exact for fp32 and for bf16 bits)."""
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    if dtype == "bf16":
+        bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+        return bits.view(np.float32).astype(np.float64)
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+def default_scale(d_h: int) -> float:
+    return 1.0 / np.sqrt(float(d_h))
+
+
+# ----------------------------------------------------------------------------
+# 8. cache size
+# ----------------------------------------------------------------------------
+def cache_bytes(L: int, S: int, n_kv: int, d_h: int, b: int) -> int:
+    """Bytes of a K+V cache for one sequence: two tensors (K and V) of
+    L layers x S tokens x n_kv heads x d_h elements x b bytes."""
+    return 2 * int(L) * int(S) * int(n_kv) * int(d_h) * int(b)
+
+
+# ----------------------------------------------------------------------------
+# 1-2. window probabilities and raw scores
+# ----------------------------------------------------------------------------
+def window_probs(q_rows: np.ndarray, k_head: np.ndarray, w: int, scale: float):
+    """Softmax rows of the observation window for one (sequence, KV head).
+
+    q_rows: [G, w, d] float64 -- the window queries of the G query heads that
+            share this KV head, row i at absolute position len - w + i.
+    k_head: [len, d] float64 -- every cached key of this KV head.
+    Returns (pi [G, w, len], m [G, w], l [G, w]) with pi zero on masked keys;
+    m is the row maximum of the visible logits and l the sum of exp(z - m).
+    """
+    G, w_, d = q_rows.shape
+    assert w_ == w
+    length = k_head.shape[0]
+    z = scale * (q_rows.reshape(G * w, d) @ k_head.T).reshape(G, w, length)
+    pos = (length - w) + np.arange(w)                        # absolute row positions
+    visible = np.arange(length)[None, :] <= pos[:, None]     # [w, len]
+    z = np.where(visible[None, :, :], z, -np.inf)
+    m = z.max(axis=2)
+    e = np.exp(z - m[:, :, None])                            # exp(-inf) = 0
+    l = e.sum(axis=2)
+    return e / l[:, :, None], m, l
+
+
+def raw_scores(q_win: np.ndarray, k: np.ndarray, cu_seqlens, n_h: int, n_kv: int, w: int,
+               dtype: str, scale: float | None = None) -> np.ndarray:
+    """raw[h, t] for every packed token t: the softmax mass that the window rows
+    of the G query heads of KV head h put on token t (window tokens included,
+    where the causal mask applies).  Shape [n_kv, T], float64.
+
+    q_win: [n_seqs * w, n_h, d] stored;  k: [T, n_kv, d] stored.
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    n_seqs = len(cu) - 1
+    d = k.shape[2]
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    G = n_h // n_kv
+    qf = to_f64(q_win, dtype)
+    kf = to_f64(k, dtype)
+    out = np.zeros((n_kv, int(cu[-1])), dtype=np.float64)
+    for b in range(n_seqs):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        qb = qf[b * w:(b + 1) * w]                            # [w, n_h, d]
+        for h in range(n_kv):
+            q_rows = np.transpose(qb[:, h * G:(h + 1) * G, :], (1, 0, 2))   # [G, w, d]
+            pi, _, _ = window_probs(q_rows, kf[t0:t1, h, :], w, scale)
+            out[h, t0:t1] = pi.sum(axis=(0, 1))
+    return out
+
+
+def row_stats(q_win: np.ndarray, k: np.ndarray, cu_seqlens, n_h: int, n_kv: int, w: int,
+              dtype: str, scale: float | None = None):
+    """(m, l) of every window row, shapes [n_seqs, n_h, w]: m = max visible
+    logit (natural-log units), l = sum over visible keys of exp(z - m)."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    n_seqs = len(cu) - 1
+    d = k.shape[2]
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    G = n_h // n_kv
+    qf = to_f64(q_win, dtype)
+    kf = to_f64(k, dtype)
+    m_all = np.zeros((n_seqs, n_h, w))
+    l_all = np.zeros((n_seqs, n_h, w))
+    for b in range(n_seqs):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        qb = qf[b * w:(b + 1) * w]
+        for h in range(n_kv):
+            q_rows = np.transpose(qb[:, h * G:(h + 1) * G, :], (1, 0, 2))
+            _, m, l = window_probs(q_rows, kf[t0:t1, h, :], w, scale)
+            m_all[b, h * G:(h + 1) * G] = m
+            l_all[b, h * G:(h + 1) * G] = l
+    return m_all, l_all
+
+
+# ----------------------------------------------------------------------------
+# 3. pooling
+# ----------------------------------------------------------------------------
+def maxpool1d_same(x: np.ndarray, pool_k: int) -> np.ndarray:
+    """out[j] = max of x[j + t] over |t| <= (pool_k - 1) / 2 with 0 <= j + t < len(x)."""
+    if pool_k < 1 or pool_k % 2 == 0:
+        raise ValueError("pool_k must be odd and >= 1")
+    r = (pool_k - 1) // 2
+    n = x.shape[0]
+    out = x.copy()
+    for t in range(1, r + 1):
+        out[:n - t] = np.maximum(out[:n - t], x[t:])        # right neighbour j + t
+        out[t:] = np.maximum(out[t:], x[:n - t])            # left neighbour j - t
+    return out
+
+
+def pool_prefix(raw: np.ndarray, cu_seqlens, w: int, pool_k: int) -> np.ndarray:
+    """Pooled scores [n_kv, T]: on each sequence's prefix [0, P) the max-pool of
+    raw over that prefix; window positions carry +inf (always retained)."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    out = np.full_like(raw, np.inf)
+    for b in range(len(cu) - 1):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        P = max(t1 - t0 - w, 0)
+        for h in range(raw.shape[0]):
+            out[h, t0:t0 + P] = maxpool1d_same(raw[h, t0:t0 + P], pool_k)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# 4. selection
+# ----------------------------------------------------------------------------
+def budget_offsets(seqlens, budget: int) -> np.ndarray:
+    """cu_budget: prefix sums of min(budget, len_b), int64, length n_seqs + 1."""
+    kept = np.minimum(np.asarray(seqlens, dtype=np.int64), int(budget))
+    out = np.zeros(len(kept) + 1, dtype=np.int64)
+    out[1:] = np.cumsum(kept)
+    return out
+
+
+def topk_prefix(scores: np.ndarray, k_sel: int) -> np.ndarray:
+    """The k_sel positions with the largest scores (ties: lower index first),
+    returned in ascending position order."""
+    order = np.argsort(-scores, kind="stable")               # descending score, index asc on ties
+    return np.sort(order[:k_sel])
+
+
+def select_one(pooled_prefix: np.ndarray, length: int, w: int, budget: int) -> np.ndarray:
+    """Retained positions of one (sequence, KV head): ascending prefix winners,
+    then the window P..len-1; all positions when budget >= len."""
+    if budget < w:
+        raise ValueError("budget must be >= w (the window is always kept)")
+    if budget >= length:
+        return np.arange(length, dtype=np.int64)
+    P = length - w
+    chosen = topk_prefix(pooled_prefix[:P], budget - w)
+    return np.concatenate([chosen, np.arange(P, length, dtype=np.int64)])
+
+
+def select_topk(pooled: np.ndarray, cu_seqlens, w: int, budget: int) -> np.ndarray:
+    """idx [n_kv, sum_b min(budget, len_b)], int64, sequence-local positions."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lens = np.diff(cu)
+    cb = budget_offsets(lens, budget)
+    n_kv = pooled.shape[0]
+    idx = np.zeros((n_kv, int(cb[-1])), dtype=np.int64)
+    for b in range(len(lens)):
+        t0 = int(cu[b])
+        for h in range(n_kv):
+            idx[h, cb[b]:cb[b + 1]] = select_one(pooled[h, t0:t0 + lens[b]], int(lens[b]), w, budget)
+    return idx
+
+
+# ----------------------------------------------------------------------------
+# 5. gather
+# ----------------------------------------------------------------------------
+def gather_kv(k: np.ndarray, v: np.ndarray, idx: np.ndarray, cu_seqlens, budget: int):
+    """K_c[cb_b + t, h] = K[cu_b + idx[h, cb_b + t], h] (same for V); any dtype,
+    bytes copied unchanged."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lens = np.diff(cu)
+    cb = budget_offsets(lens, budget)
+    n_kv = k.shape[1]
+    kc = np.empty((int(cb[-1]),) + k.shape[1:], dtype=k.dtype)
+    vc = np.empty_like(kc)
+    for b in range(len(lens)):
+        for h in range(n_kv):
+            src = cu[b] + idx[h, cb[b]:cb[b + 1]]
+            kc[cb[b]:cb[b + 1], h] = k[src, h]
+            vc[cb[b]:cb[b + 1], h] = v[src, h]
+    return kc, vc
+
+
+# ----------------------------------------------------------------------------
+# 6. decode attention
+# ----------------------------------------------------------------------------
+def gqa_decode(q: np.ndarray, k_c: np.ndarray, v_c: np.ndarray, row_offset, kv_len,
+               n_kv: int, dtype: str, scale: float | None = None) -> np.ndarray:
+    """out[b, qh] = sum_t softmax_t(scale * q[b, qh] . K_c[off_b + t, qh // G]) V_c[off_b + t, qh // G]
+    over t < kv_len[b]; an empty cache gives 0.  float64 [batch, n_h, d]."""
+    qf = to_f64(q, dtype)
+    kf = to_f64(k_c, dtype)
+    vf = to_f64(v_c, dtype)
+    batch, n_h, d = qf.shape
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    G = n_h // n_kv
+    out = np.zeros((batch, n_h, d))
+    for b in range(batch):
+        o, n = int(row_offset[b]), int(kv_len[b])
+        if n == 0:
+            continue
+        for qh in range(n_h):
+            h = qh // G
+            z = scale * (kf[o:o + n, h, :] @ qf[b, qh])
+            e = np.exp(z - z.max())
+            out[b, qh] = (e / e.sum()) @ vf[o:o + n, h, :]
+    return out
+
+
+# ----------------------------------------------------------------------------
+# 7. FastKV token-selective propagation
+# ----------------------------------------------------------------------------
+def tsp_select(raw: np.ndarray, S: int, w: int, pool_k: int, k_tsp: int) -> np.ndarray:
+    """One token set for the layer: the k_tsp prefix positions with the largest
+    pooled head-summed score (ties: lower index), ascending, then the window.
+
+    raw: [n_rows, S] per-head raw scores of one sequence (rows summed here)."""
+    P = S - w
+    if k_tsp < 0 or k_tsp > P:
+        raise ValueError("k_tsp must lie in [0, S - w]")
+    agg = raw[:, :P].sum(axis=0)
+    pooled = maxpool1d_same(agg, pool_k)
+    chosen = topk_prefix(pooled, k_tsp)
+    return np.concatenate([chosen, np.arange(P, S, dtype=np.int64)])
+
+
+def tsp_pooled(raw: np.ndarray, S: int, w: int, pool_k: int) -> np.ndarray:
+    P = S - w
+    return maxpool1d_same(raw[:, :P].sum(axis=0), pool_k)
+
+
+def tsp_gather(hidden: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """Propagated hidden states: hidden rows idx, bytes unchanged."""
+    return hidden[np.asarray(idx, dtype=np.int64)].copy()
+
+
+def rate_count(rate: float, S: int) -> int:
+    """Token count of a rate applied to S tokens (reading: floor)."""
+    return int(np.floor(rate * S))

@@ -1,0 +1,360 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself:
+the pages' worked example, closed forms, invariants, brute force on tiny
+inputs, and library routines for the special cases that reduce to them."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvc_oracle as O
+from kv_cache_compression_score_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f32(a):
+    return np.asarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------------------
+# cache-size formula: the pages' worked example
+# ---------------------------------------------------------------------------
+def test_cache_bytes_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "cache_bytes.json")))
+    for c in g["cases"]:
+        n = c.get("n_seqs", 1)
+        assert n * O.cache_bytes(c["L"], c["S"], c["n_kv"], c["d_h"], c["b"]) == c["bytes"], c["what"]
+    wk = g["weak"]
+    assert O.cache_bytes(wk["L"], wk["S"], wk["n_kv"], wk["d_h"], wk["b"]) == wk["gib"] * 2**30
+
+
+# ---------------------------------------------------------------------------
+# scoring: closed forms
+# ---------------------------------------------------------------------------
+def _batch(lengths, n_h, n_kv, d, w, seed=7, dtype="f32"):
+    return synth.packed_batch(seed, lengths, n_h, n_kv, d, w, dtype)
+
+
+@pytest.mark.parametrize("lengths,n_h,n_kv,w", [([40], 4, 2, 5), ([33, 17, 9], 6, 3, 4), ([12], 2, 2, 12)])
+def test_zero_keys_closed_form(lengths, n_h, n_kv, w):
+    """K = 0: every visible logit is 0, so row i spreads 1/(P+i+1) over its
+    P+i+1 visible keys; raw is G * sum_{i >= max(0, j-P)} 1/(P+i+1)."""
+    d = 8
+    bt = _batch(lengths, n_h, n_kv, d, w)
+    k = np.zeros_like(bt["k"])
+    raw = O.raw_scores(bt["q_win"], k, bt["cu_seqlens"], n_h, n_kv, w, "f32")
+    G = n_h // n_kv
+    for b, L in enumerate(lengths):
+        t0 = bt["cu_seqlens"][b]
+        P = L - w
+        for j in range(L):
+            first_row = max(0, j - P)
+            expect = G * sum(1.0 / (P + i + 1) for i in range(first_row, w))
+            np.testing.assert_allclose(raw[:, t0 + j], expect, rtol=1e-13)
+    # Q = 0 gives the same closed form
+    raw_q0 = O.raw_scores(np.zeros_like(bt["q_win"]), bt["k"], bt["cu_seqlens"], n_h, n_kv, w, "f32")
+    np.testing.assert_allclose(raw_q0, raw, rtol=1e-13)
+
+
+def test_row_stats_zero_keys():
+    """K = 0: m = 0 and l = number of visible keys = P + i + 1."""
+    L, w, n_h, n_kv = 30, 6, 4, 2
+    bt = _batch([L], n_h, n_kv, 8, w)
+    m, l = O.row_stats(bt["q_win"], np.zeros_like(bt["k"]), bt["cu_seqlens"], n_h, n_kv, w, "f32")
+    assert np.all(m == 0.0)
+    np.testing.assert_array_equal(l[0], np.broadcast_to(L - w + 1 + np.arange(w), (n_h, w)))
+
+
+def test_scale_two_key_closed_form():
+    """One row, two visible keys: z1 = scale*a, z2 = 0, so p1 = 1/(1+exp(-scale*a))."""
+    d, a, scale = 4, 3.0, 0.37
+    q = np.zeros((1, 1, d)); q[0, 0, 0] = a
+    k = np.zeros((2, d)); k[0, 0] = 1.0
+    pi, m, l = O.window_probs(q, k, 1, scale)
+    np.testing.assert_allclose(pi[0, 0, 0], 1.0 / (1.0 + math.exp(-scale * a)), rtol=1e-15)
+    np.testing.assert_allclose(m[0, 0], scale * a, rtol=1e-15)
+
+
+def test_probability_mass_invariant():
+    """Each window row is a probability distribution: summed over all visible
+    keys (prefix and window) the raw scores of a KV head total G * w."""
+    lengths, n_h, n_kv, w = [70, 41], 8, 2, 6
+    bt = _batch(lengths, n_h, n_kv, 16, w, seed=3)
+    raw = O.raw_scores(bt["q_win"], bt["k"], bt["cu_seqlens"], n_h, n_kv, w, "f32")
+    cu = bt["cu_seqlens"]
+    for b in range(len(lengths)):
+        s = raw[:, cu[b]:cu[b + 1]].sum(axis=1)
+        np.testing.assert_allclose(s, (n_h // n_kv) * w, rtol=1e-12)
+
+
+def test_brute_force_loops_tiny():
+    """Pure-Python loops (math.exp, explicit causal test) on a tiny ragged batch."""
+    lengths, n_h, n_kv, w, d = [9, 6], 4, 2, 3, 5
+    bt = _batch(lengths, n_h, n_kv, d, w, seed=11)
+    scale = 0.41
+    raw = O.raw_scores(bt["q_win"], bt["k"], bt["cu_seqlens"], n_h, n_kv, w, "f32", scale)
+    q = bt["q_win"].astype(np.float64)
+    k = bt["k"].astype(np.float64)
+    G = n_h // n_kv
+    for b, L in enumerate(lengths):
+        t0 = int(bt["cu_seqlens"][b])
+        for h in range(n_kv):
+            acc = [0.0] * L
+            for g in range(G):
+                for i in range(w):
+                    row_pos = L - w + i
+                    zs = []
+                    for j in range(L):
+                        if j <= row_pos:
+                            zs.append(scale * sum(q[b * w + i, h * G + g, e] * k[t0 + j, h, e] for e in range(d)))
+                    mx = max(zs)
+                    den = sum(math.exp(z - mx) for z in zs)
+                    for j, z in enumerate(zs):
+                        acc[j] += math.exp(z - mx) / den
+            np.testing.assert_allclose(raw[h, t0:t0 + L], acc, rtol=1e-12)
+
+
+def test_gqa_contiguous_mapping():
+    """Query heads 0..G-1 use KV head 0 (contiguous groups).  Heads of group 0
+    point at a spike key of KV head 0 only; group 1 at a spike of KV head 1."""
+    L, w, d, n_h, n_kv = 40, 4, 8, 4, 2
+    k = np.zeros((L, n_kv, d), dtype=np.float32)
+    k[5, 0, 0] = 30.0            # spike of KV head 0 along e0
+    k[20, 1, 1] = 30.0           # spike of KV head 1 along e1
+    q = np.zeros((w, n_h, d), dtype=np.float32)
+    q[:, 0:2, 0] = 1.0           # group 0 -> e0
+    q[:, 2:4, 1] = 1.0           # group 1 -> e1
+    raw = O.raw_scores(q, k, np.array([0, L]), n_h, n_kv, w, "f32", scale=1.0)
+    assert raw[0, 5] > 0.99 * 2 * w and raw[1, 20] > 0.99 * 2 * w
+    assert raw[0, 20] < 0.01 and raw[1, 5] < 0.01
+
+
+# ---------------------------------------------------------------------------
+# pooling
+# ---------------------------------------------------------------------------
+def test_pool_matches_torch_maxpool():
+    x = synth.random_scores(5, (300,)).astype(np.float64)
+    for pk in (1, 3, 7, 9):
+        ref = torch.nn.functional.max_pool1d(torch.tensor(x)[None, None], pk, stride=1,
+                                             padding=(pk - 1) // 2)[0, 0].numpy()
+        np.testing.assert_array_equal(O.maxpool1d_same(x, pk), ref)
+
+
+def test_spike_plateau_and_window_excluded():
+    """A dominant prefix key j* gives a pooled plateau of width 7 (clipped to the
+    prefix); a dominant window key does not leak into the pooled prefix."""
+    L, w, d, n_h, n_kv, pk = 64, 8, 8, 2, 1, 7
+    P = L - w
+    for jstar in (0, 2, 30, P - 2, P - 1):
+        k = np.zeros((L, n_kv, d), dtype=np.float32)
+        k[jstar, 0, 0] = 40.0
+        q = np.zeros((w, n_h, d), dtype=np.float32); q[:, :, 0] = 1.0
+        cu = np.array([0, L])
+        raw = O.raw_scores(q, k, cu, n_h, n_kv, w, "f32", scale=1.0)
+        pooled = O.pool_prefix(raw, cu, w, pk)
+        hot = np.where(pooled[0, :P] > 0.9 * n_h * w)[0]
+        np.testing.assert_array_equal(hot, np.arange(max(0, jstar - 3), min(P, jstar + 4)))
+        assert np.all(np.isinf(pooled[0, P:]))
+    # spike on the first window key: visible to every window row, never pooled into the prefix
+    k = np.zeros((L, n_kv, d), dtype=np.float32); k[P, 0, 0] = 40.0
+    q = np.zeros((w, n_h, d), dtype=np.float32); q[:, :, 0] = 1.0
+    raw = O.raw_scores(q, k, np.array([0, L]), n_h, n_kv, w, "f32", scale=1.0)
+    pooled = O.pool_prefix(raw, np.array([0, L]), w, pk)
+    assert raw[0, P] > 0.99 * n_h * w
+    assert pooled[0, :P].max() < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# selection
+# ---------------------------------------------------------------------------
+def _brute_topk(scores, k_sel):
+    """Among all k_sel-subsets: maximise the descending score vector, then take
+    the lexicographically smallest index tuple (lowest-index tie rule)."""
+    best_key, best = None, None
+    for sub in itertools.combinations(range(len(scores)), k_sel):
+        key = (tuple(sorted((scores[i] for i in sub), reverse=True)), tuple(-i for i in sub))
+        if best_key is None or key > best_key:
+            best_key, best = key, sub
+    return np.array(best, dtype=np.int64)
+
+
+def test_topk_brute_force_with_ties():
+    for seed in range(12):
+        n = 6 + seed % 7
+        s = synth.random_scores(seed, (n,), n_levels=3).astype(np.float64)
+        for k_sel in range(0, n + 1):
+            np.testing.assert_array_equal(O.topk_prefix(s, k_sel), _brute_topk(s, k_sel))
+
+
+def test_select_one_brute_force():
+    for seed in range(8):
+        L, w = 9 + seed % 5, 2 + seed % 2
+        s = synth.random_scores(100 + seed, (L,), n_levels=4).astype(np.float64)
+        pooled = O.maxpool1d_same(s[:L - w], 3)
+        for budget in range(w, L + 2):
+            got = O.select_one(pooled, L, w, budget)
+            if budget >= L:
+                np.testing.assert_array_equal(got, np.arange(L))
+                continue
+            expect = np.concatenate([_brute_topk(pooled, budget - w), np.arange(L - w, L)])
+            np.testing.assert_array_equal(got, expect)
+
+
+def test_select_invariants_and_edges():
+    lengths, n_h, n_kv, w, B = [50, 33, 12], 4, 2, 6, 20
+    bt = _batch(lengths, n_h, n_kv, 8, w, seed=21)
+    cu = bt["cu_seqlens"]
+    raw = O.raw_scores(bt["q_win"], bt["k"], cu, n_h, n_kv, w, "f32")
+    pooled = O.pool_prefix(raw, cu, w, 7)
+    idx = O.select_topk(pooled, cu, w, B)
+    cb = O.budget_offsets(lengths, B)
+    assert idx.shape == (n_kv, cb[-1])
+    for b, L in enumerate(lengths):
+        seg = idx[:, cb[b]:cb[b + 1]]
+        for h in range(n_kv):
+            assert np.all(np.diff(seg[h]) > 0)                      # ascending, distinct
+            assert set(range(L - w, L)) <= set(seg[h].tolist())     # window always kept
+            if B >= L:
+                np.testing.assert_array_equal(seg[h], np.arange(L))
+    # all scores equal (K = 0): the lowest prefix positions win
+    raw0 = O.raw_scores(bt["q_win"], np.zeros_like(bt["k"]), cu, n_h, n_kv, w, "f32")
+    idx0 = O.select_topk(O.pool_prefix(raw0, cu, w, 7), cu, w, B)
+    np.testing.assert_array_equal(idx0[0, :B], np.concatenate([np.arange(B - w), np.arange(50 - w, 50)]))
+    with pytest.raises(ValueError):
+        O.select_one(np.zeros(10), 14, 4, 3)
+    with pytest.raises(ValueError):
+        O.maxpool1d_same(np.zeros(5), 4)
+
+
+# ---------------------------------------------------------------------------
+# gather + decode
+# ---------------------------------------------------------------------------
+def test_gather_bytes_and_identity():
+    lengths, n_kv, w, B = [20, 7], 2, 3, 10
+    bt = _batch(lengths, 4, n_kv, 8, w, seed=5, dtype="bf16")
+    cu = bt["cu_seqlens"]
+    idx = np.concatenate([np.stack([np.arange(10)[::-1] % 20] * n_kv), np.stack([np.arange(7)] * n_kv)], axis=1)
+    kc, vc = O.gather_kv(bt["k"], bt["v"], idx, cu, B)
+    assert kc.dtype == np.uint16
+    for t in range(10):
+        np.testing.assert_array_equal(kc[t], bt["k"][idx[0, t]])
+    np.testing.assert_array_equal(kc[10:], bt["k"][20:27])
+    np.testing.assert_array_equal(vc[10:], bt["v"][20:27])
+
+
+def test_decode_closed_forms():
+    n_h, n_kv, d, n = 4, 2, 8, 13
+    q = synth.decode_queries(1, 1, n_h, d, "f32")
+    rng_k, rng_v = synth.keys_values(2, 0, n, n_kv, d, "f32")
+    off, ln = np.array([0]), np.array([n])
+    # equal V rows -> that row
+    v_eq = np.broadcast_to(rng_v[3:4], rng_v.shape).copy()
+    out = O.gqa_decode(q, rng_k, v_eq, off, ln, n_kv, "f32")
+    for qh in range(n_h):
+        np.testing.assert_allclose(out[0, qh], rng_v[3, qh // 2].astype(np.float64), rtol=1e-14)
+    # K = 0 -> mean of V
+    out = O.gqa_decode(q, np.zeros_like(rng_k), rng_v, off, ln, n_kv, "f32")
+    for qh in range(n_h):
+        np.testing.assert_allclose(out[0, qh], rng_v[:, qh // 2].astype(np.float64).mean(0), rtol=1e-12)
+    # permuting cache rows leaves the output unchanged
+    perm = np.array(synth.boosted_positions(9, 0, 0, n, 1.0))[::-1]
+    a = O.gqa_decode(q, rng_k, rng_v, off, ln, n_kv, "f32")
+    b = O.gqa_decode(q, rng_k[perm], rng_v[perm], off, ln, n_kv, "f32")
+    np.testing.assert_allclose(a, b, rtol=1e-12)
+    # two rows, closed form with the scale
+    k2 = np.zeros((2, 1, 2), dtype=np.float32); k2[0, 0, 0] = 1.0
+    v2 = np.zeros((2, 1, 2), dtype=np.float32); v2[0, 0, 1] = 1.0; v2[1, 0, 0] = 1.0
+    q2 = np.zeros((1, 1, 2), dtype=np.float32); q2[0, 0, 0] = 2.0
+    o2 = O.gqa_decode(q2, k2, v2, [0], [2], 1, "f32", scale=0.5)
+    p0 = 1.0 / (1.0 + math.exp(-1.0))
+    np.testing.assert_allclose(o2[0, 0], [1 - p0, p0], rtol=1e-15)
+    # empty cache -> 0
+    assert np.all(O.gqa_decode(q, rng_k, rng_v, off, np.array([0]), n_kv, "f32") == 0)
+
+
+def test_decode_matches_torch_sdpa_and_identity_budget():
+    """B >= S: selection is the identity and decode over the compact cache
+    equals full attention (torch fp64 scaled_dot_product_attention)."""
+    L, n_h, n_kv, d, w = 37, 8, 2, 16, 4
+    bt = _batch([L], n_h, n_kv, d, w, seed=31, dtype="bf16")
+    cu = bt["cu_seqlens"]
+    raw = O.raw_scores(bt["q_win"], bt["k"], cu, n_h, n_kv, w, "bf16")
+    idx = O.select_topk(O.pool_prefix(raw, cu, w, 7), cu, w, L + 5)
+    np.testing.assert_array_equal(idx, np.broadcast_to(np.arange(L), (n_kv, L)))
+    kc, vc = O.gather_kv(bt["k"], bt["v"], idx, cu, L + 5)
+    np.testing.assert_array_equal(kc, bt["k"])
+    q = synth.decode_queries(4, 1, n_h, d, "bf16")
+    out = O.gqa_decode(q, kc, vc, [0], [L], n_kv, "bf16")
+    G = n_h // n_kv
+    qt = torch.tensor(O.to_f64(q, "bf16"))[:, :, None, :]                       # [1, n_h, 1, d]
+    kt = torch.tensor(O.to_f64(bt["k"], "bf16")).permute(1, 0, 2).repeat_interleave(G, 0)[None]
+    vt = torch.tensor(O.to_f64(bt["v"], "bf16")).permute(1, 0, 2).repeat_interleave(G, 0)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)[0, :, 0].numpy()
+    np.testing.assert_allclose(out[0], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_window_probs_match_torch_softmax():
+    """The causal window softmax is torch's fp64 softmax over the visible keys."""
+    bt = _batch([25], 4, 2, 8, 5, seed=41)
+    qf = O.to_f64(bt["q_win"], "f32"); kf = O.to_f64(bt["k"], "f32")
+    pi, _, _ = O.window_probs(np.transpose(qf[:, 0:2], (1, 0, 2)), kf[:, 0], 5, 0.3)
+    z = 0.3 * torch.einsum("igd,jd->gij", torch.tensor(qf[:, 0:2]), torch.tensor(kf[:, 0]))
+    mask = torch.ones(5, 25, dtype=torch.bool).tril(diagonal=20)
+    ref = torch.softmax(z.masked_fill(~mask, float("-inf")), dim=-1).numpy()
+    np.testing.assert_allclose(pi, ref, rtol=1e-13, atol=1e-300)
+
+
+# ---------------------------------------------------------------------------
+# TSP
+# ---------------------------------------------------------------------------
+def test_tsp_rates_and_ties():
+    assert O.rate_count(0.2, 32768) == 6553
+    assert O.rate_count(0.1, 32768) == 3276
+    S, w = 40, 4
+    raw = np.ones((3, S))
+    idx = O.tsp_select(raw, S, w, 7, 10)
+    np.testing.assert_array_equal(idx, np.concatenate([np.arange(10), np.arange(36, 40)]))
+    with pytest.raises(ValueError):
+        O.tsp_select(raw, S, w, 7, S - w + 1)
+
+
+def test_tsp_sums_heads_before_pooling():
+    """Disjoint spikes in different heads both survive the head sum; a spike
+    smaller than another head's plateau still wins where it is alone."""
+    S, w = 60, 4
+    raw = np.zeros((2, S))
+    raw[0, 10] = 5.0
+    raw[1, 40] = 3.0
+    pooled = O.tsp_pooled(raw, S, w, 3)
+    np.testing.assert_array_equal(np.where(pooled == 5.0)[0], [9, 10, 11])
+    np.testing.assert_array_equal(np.where(pooled == 3.0)[0], [39, 40, 41])
+    idx = O.tsp_select(raw, S, w, 3, 6)
+    np.testing.assert_array_equal(idx, [9, 10, 11, 39, 40, 41, 56, 57, 58, 59])
+    hidden = synth.hidden_states(3, S, 16, "bf16")
+    np.testing.assert_array_equal(O.tsp_gather(hidden, idx), hidden[idx])
+    # two heads agreeing on a moderate token outrank one head's larger spike
+    raw = np.zeros((2, S))
+    raw[0, 20] = raw[1, 20] = 3.0
+    raw[0, 45] = 5.0
+    np.testing.assert_array_equal(O.tsp_select(raw, S, w, 1, 1), [20, 56, 57, 58, 59])
+
+
+# ---------------------------------------------------------------------------
+# generator sanity (inputs, not the method)
+# ---------------------------------------------------------------------------
+def test_generators_deterministic_and_normal():
+    a = synth.normal_tensor(1, synth.T_K, 0, (1000, 4), "f32")
+    b = synth.normal_tensor(1, synth.T_K, 0, (1000, 4), "f32")
+    np.testing.assert_array_equal(a, b)
+    assert abs(a.mean()) < 0.05 and abs(a.std() - 1) < 0.05
+    bits = synth.normal_tensor(1, synth.T_K, 0, (1000, 4), "bf16")
+    back = synth.bf16_bits_to_f32(bits)
+    assert np.max(np.abs(back - a) / np.maximum(np.abs(a), 1e-30)) <= 2.0 ** -8
+    lens = synth.ragged_lengths(1005, 16, 4096, 65536)
+    assert lens.min() >= 4096 and lens.max() <= 65536
+    pos = synth.boosted_positions(1002, 0, 0, 32768, 0.01)
+    assert len(pos) == 327 and len(np.unique(pos)) == 327
