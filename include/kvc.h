@@ -1,0 +1,200 @@
+/*
+ * kvc.h -- C ABI of libkvc, the B200 (sm_100a) hot path of observation-window
+ * KV-cache compression: window saliency scoring, budgeted per-KV-head top-k,
+ * compact KV gather, GQA decode attention over the compact cache, and
+ * FastKV-style token-selective propagation (TSP).
+ *
+ * Sources of the method (web pages; the library implements their outline and
+ * states its readings of the points they leave open):
+ *   - "Variantes de l'attention et compression du cache KV" (nickwang.xyz):
+ *     section "MHA et GQA" (head sharing, cache-size formula), section
+ *     "Quand la reutilisation est-elle exacte ?" (causal offset of appended
+ *     rows; original positions kept after eviction), section "Compresser un
+ *     cache existant" (SnapKV observation-window scoring; sliding windows keep
+ *     a recent region).
+ *   - "FastKV: Decoupling of Context Reduction and KV Cache Compression for
+ *     Prefill-Decoding Acceleration" (gist.science 2502.01068): section 2.A
+ *     (token-selective propagation from window-attention saliency), section
+ *     2.B (TSP rate independent of the KV retention rate).
+ *   - "FreeKV: Boosting KV Cache Retrieval for Efficient LLM Inference"
+ *     (gist.science 2505.13109), technical summary section 2.B: NHD layout on
+ *     the GPU, which every cache tensor here uses.
+ *
+ * Conventions shared by every entry point
+ *   - All calls are asynchronous on the caller's stream (a cudaStream_t passed
+ *     as kvc_stream_t; NULL is the legacy default stream).  No call allocates,
+ *     frees or synchronises; no call reads device memory on the host.
+ *   - The caller owns every buffer.  Device pointers must be 16-byte aligned
+ *     and dense in the layouts stated below.  Host pointers are read during the
+ *     call only.
+ *   - Scratch memory is a caller-provided device workspace whose size comes
+ *     from the matching *_workspace_size() query; it may be reused between
+ *     calls on the same stream.  The decode workspace holds completion
+ *     counters that must be zero before its first use (cudaMemset to 0 once);
+ *     every decode call leaves them zero again.
+ *   - Ragged batches: n_seqs sequences packed along the token axis; seqlens_host
+ *     (host int32[n_seqs]) gives the lengths, cu_seqlens (device int32[n_seqs+1])
+ *     their prefix sums starting at 0.  Both must describe the same batch.
+ *   - Layouts: K, V, compact K_c/V_c: [rows, n_kv, d_h] (NHD).  Window queries
+ *     q_win: [n_seqs * w, n_h, d_h], the last w query rows of each sequence in
+ *     order.  Scores: float32 [n_kv, T], T = sum of lengths.  Index lists:
+ *     int32 [n_kv, sum_b min(budget, len_b)], sequence b's segment starting at
+ *     cu_budget[b].
+ *   - GQA: query head qh attends with KV head qh / (n_h / n_kv).
+ *   - scale <= 0 selects 1/sqrt(d_h).
+ *   - Errors: validation failures return before anything is launched and set a
+ *     thread-local message readable with kvc_last_error().  A failed launch
+ *     returns KVC_ERR_CUDA; work already enqueued by that call is not undone.
+ */
+#ifndef KVC_H_
+#define KVC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvc_stream_t; /* identical to cudaStream_t */
+
+typedef enum kvc_status {
+  KVC_OK = 0,
+  KVC_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or count */
+  KVC_ERR_UNSUPPORTED = 2,  /* valid request outside the kernels' shapes/dtypes */
+  KVC_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  KVC_ERR_CUDA = 4          /* a CUDA runtime call or launch failed */
+} kvc_status;
+
+typedef enum kvc_dtype {
+  KVC_F32 = 0,   /* IEEE binary32 */
+  KVC_BF16 = 1   /* bfloat16 */
+} kvc_dtype;
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int kvc_version(void);
+
+/* Static text for a status code. */
+const char *kvc_status_string(int status);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char *kvc_last_error(void);
+
+/*
+ * Bytes of a K+V cache for one sequence: 2 * L * S * n_kv * d_h * b.
+ * The factor 2 counts keys and values ("MHA et GQA" on the attention-variants
+ * page; its worked example L=32, S=4096, n_kv=8, d_h=128, b=2 gives
+ * 536,870,912).  Returns 0 if an argument is negative.  Host only.
+ */
+uint64_t kvc_cache_bytes(int L, int64_t S, int n_kv, int d_h, int b);
+
+/*
+ * Host helper: cu_budget_host[0] = 0, cu_budget_host[b+1] = cu_budget_host[b]
+ * + min(budget, seqlens_host[b]).  cu_budget_host has n_seqs + 1 entries.
+ * Returns the total (the compact-cache row count) or -1 on invalid input.
+ */
+int64_t kvc_budget_offsets(int n_seqs, const int32_t *seqlens_host, int budget,
+                           int32_t *cu_budget_host);
+
+/* ------------------------------------------------------------------------
+ * Window saliency scores (SnapKV observation window; FastKV 2.A saliency).
+ *
+ * For sequence b (length len_b >= w, prefix P_b = len_b - w), KV head h,
+ * query head g of h's group and window row i (position P_b + i), with logits
+ * z_j = scale * q . k_j over the visible keys j <= P_b + i (causal rule of the
+ * attention-variants page, "Quand la reutilisation est-elle exacte ?"):
+ *   raw[h][t0 + j]    = sum_{g, i} softmax_j(z)      for every j < len_b
+ *   scores[h][t0 + j] = max_{|t| <= r, 0 <= j+t < P_b} raw[h][t0 + j + t]
+ *                       for j < P_b (r = (pool_k - 1) / 2), and +inf on the
+ *                       window positions j >= P_b (always retained).
+ * The softmax is exact (two passes over K: row max/sum, then probabilities).
+ *
+ * dt: KVC_F32 or KVC_BF16 for q_win and k.  d_h in {64, 128}.  n_h % n_kv == 0,
+ * G = n_h / n_kv; the window block has G * w <= 256 rows (and a multiple of 16
+ * rows for KVC_BF16).  pool_k odd in [1, 31].  scores_raw may be NULL.
+ * q_win: [n_seqs * w, n_h, d_h];  k: [T, n_kv, d_h];  scores, scores_raw:
+ * float32 [n_kv, T].  ws: kvc_score_window_workspace_size() bytes.
+ * ------------------------------------------------------------------------ */
+size_t kvc_score_window_workspace_size(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host,
+                                       int n_h, int n_kv, int d_h, int w);
+kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host,
+                            const int32_t *cu_seqlens, int n_h, int n_kv, int d_h, int w,
+                            int pool_k, float scale, const void *q_win, const void *k,
+                            float *scores, float *scores_raw, void *ws, size_t ws_bytes,
+                            kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Budgeted per-KV-head top-k (SnapKV keeps a chosen subset; the recent window
+ * is always kept, as a sliding window keeps its recent region).
+ *
+ * For sequence b and KV head h: if budget >= len_b the segment is 0..len_b-1.
+ * Otherwise it holds the budget - w prefix positions with the largest
+ * scores[h][t0 + j], j < P_b (ties: lower position first), in ascending order,
+ * followed by P_b .. len_b - 1.  Positions are sequence-local originals
+ * (never renumbered).  Scores are compared as float32 with NaN above +inf.
+ *
+ * budget >= w >= 1.  cu_budget: device int32[n_seqs + 1] from
+ * kvc_budget_offsets().  scores: float32 [n_kv, T] (as written by
+ * kvc_score_window).  idx: int32 [n_kv, cu_budget[n_seqs]].
+ * ------------------------------------------------------------------------ */
+kvc_status kvc_select_topk(int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                           const int32_t *cu_budget, int n_kv, int w, int budget,
+                           const float *scores, int32_t *idx, kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Compact cache gather: for each sequence b, KV head h and slot t <
+ * min(budget, len_b):  K_c[cb_b + t][h][:] = K[t0_b + idx[h][cb_b + t]][h][:]
+ * and likewise for V (bytes copied unchanged).
+ *
+ * k, v: [T, n_kv, d_h];  k_out, v_out: [cu_budget[n_seqs], n_kv, d_h];  idx
+ * as written by kvc_select_topk (every entry must lie in [0, len_b)).
+ * ------------------------------------------------------------------------ */
+kvc_status kvc_gather_kv(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host,
+                         const int32_t *cu_seqlens, const int32_t *cu_budget, int n_kv, int d_h,
+                         int budget, const int32_t *idx, const void *k, const void *v,
+                         void *k_out, void *v_out, kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * FastKV token-selective propagation for one sequence of S tokens (FastKV
+ * 2.A; its rate is independent of the KV budget, 2.B):
+ *   agg[j]    = sum_{r < n_rows} scores_raw[r][j]          for j < P = S - w
+ *   pooled[j] = max_{|t| <= (pool_k-1)/2, 0 <= j+t < P} agg[j + t]
+ *   idx_out   = the k_tsp prefix positions with the largest pooled value
+ *               (ties: lower position), ascending, then P .. S-1
+ *   hidden_out[t][:] = hidden[idx_out[t]][:]   (k_tsp + w rows of D elements)
+ * scores_raw: float32 [n_rows, S] (the raw output of kvc_score_window for one
+ * sequence; summing its KV-head rows sums all query heads).  hidden: [S, D] of
+ * dt, D % 8 == 0.  idx_out: int32 [k_tsp + w].  0 <= k_tsp <= S - w.
+ * ws: kvc_tsp_workspace_size() bytes.
+ * ------------------------------------------------------------------------ */
+size_t kvc_tsp_workspace_size(int S, int w);
+kvc_status kvc_tsp_select_gather(kvc_dtype dt, int S, int n_rows, int w, int pool_k, int k_tsp,
+                                 const float *scores_raw, const void *hidden, int D,
+                                 int32_t *idx_out, void *hidden_out, void *ws, size_t ws_bytes,
+                                 kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * GQA decode attention over compact caches (decode reads the whole cache per
+ * step: FastKV section 1; attention-variants page introduction):
+ *   out[b][qh][:] = sum_{t < kv_len[b]} softmax_t(scale * q[b][qh] . Kc[o_b + t][h])
+ *                   * Vc[o_b + t][h],   h = qh / G,  o_b = kv_row_offset[b]
+ * and 0 when kv_len[b] == 0.  Offsets may alias (several queries on one cache).
+ *
+ * q: [batch, n_h, d_h] of dt;  k_c, v_c: [rows, n_kv, d_h] of dt;
+ * kv_row_offset: device int64[batch];  kv_len: device int32[batch], each
+ * <= max_kv_len;  out: float32 [batch, n_h, d_h].  G in {1, 2, 4, 8};
+ * d_h in {64, 128}.  ws: kvc_gqa_decode_workspace_size() bytes, counters
+ * zeroed before first use (see conventions).
+ * ------------------------------------------------------------------------ */
+size_t kvc_gqa_decode_workspace_size(int batch, int n_h, int n_kv, int d_h, int max_kv_len);
+kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, float scale,
+                               const void *q, const void *k_c, const void *v_c,
+                               const int64_t *kv_row_offset, const int32_t *kv_len,
+                               int max_kv_len, float *out, void *ws, size_t ws_bytes,
+                               kvc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H_ */

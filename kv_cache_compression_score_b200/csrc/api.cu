@@ -1,0 +1,333 @@
+// C ABI of libkvc: argument validation, work plans, workspace layout and
+// kernel launches.  Declarations and contracts are in include/kvc.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "kvc_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+kvc_status fail(kvc_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+kvc_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(KVC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int elem_size(kvc_dtype dt) { return dt == KVC_F32 ? 4 : dt == KVC_BF16 ? 2 : 0; }
+
+constexpr size_t kErrWordBytes = 256;   // workspace head: device error word
+
+// ------------------------------------------------------------ batch checks
+struct Batch {
+  int64_t T = 0;
+  int max_len = 0;
+  int min_len = 0;
+};
+
+kvc_status check_batch(int n_seqs, const int32_t *seqlens_host, int min_each, Batch *bt) {
+  if (n_seqs < 1) return fail(KVC_ERR_INVALID_ARG, "n_seqs must be >= 1 (got %d)", n_seqs);
+  if (!seqlens_host) return fail(KVC_ERR_INVALID_ARG, "seqlens_host is NULL");
+  int64_t T = 0;
+  int mx = 0, mn = INT32_MAX;
+  for (int b = 0; b < n_seqs; ++b) {
+    const int L = seqlens_host[b];
+    if (L < min_each) return fail(KVC_ERR_INVALID_ARG, "seqlens_host[%d] = %d is below %d", b, L, min_each);
+    T += L;
+    mx = std::max(mx, L);
+    mn = std::min(mn, L);
+  }
+  if (T >= (int64_t)INT32_MAX) return fail(KVC_ERR_INVALID_ARG, "total tokens %lld exceed int32", (long long)T);
+  bt->T = T;
+  bt->max_len = mx;
+  bt->min_len = mn;
+  return KVC_OK;
+}
+
+// --------------------------------------------------------- scoring plan
+struct ScorePlan {
+  bool tc = false;
+  int R = 0, R_pad = 0, tile = 0, keys_per_chunk = 0, n_chunks = 0;
+  Batch bt;
+  size_t off_part = 0, off_raw = 0, bytes = 0;
+};
+
+kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w,
+                      ScorePlan *pl) {
+  if (dt != KVC_F32 && dt != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+  if (n_h < 1 || n_kv < 1 || n_h % n_kv != 0)
+    return fail(KVC_ERR_INVALID_ARG, "n_h (%d) must be a positive multiple of n_kv (%d)", n_h, n_kv);
+  if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
+  if (w < 1) return fail(KVC_ERR_INVALID_ARG, "w must be >= 1 (got %d)", w);
+  const int G = n_h / n_kv;
+  if ((int64_t)G * w > 256) return fail(KVC_ERR_UNSUPPORTED, "window block G*w = %d exceeds 256 rows", G * w);
+  kvc_status s = check_batch(n_seqs, seqlens_host, w, &pl->bt);
+  if (s != KVC_OK) return s;
+  pl->R = G * w;
+  pl->tc = (dt == KVC_BF16) && pl->R <= 128;
+  pl->R_pad = pl->tc ? 128 : (pl->R + 63) / 64 * 64;
+  pl->tile = pl->tc ? kvc::tc_keys_per_tile() : kvc::simt_keys_per_tile();
+  // chunk the keys of every (sequence, head) so that about one wave of CTAs
+  // covers the batch: the smallest tiles-per-chunk whose CTA count fits
+  const int target = pl->tc ? kvc::kNumSMs : 2 * kvc::kNumSMs;
+  int64_t total_tiles = 0;
+  int max_tiles = 0;
+  std::vector<int> tiles(n_seqs);
+  for (int b = 0; b < n_seqs; ++b) {
+    tiles[b] = (seqlens_host[b] + pl->tile - 1) / pl->tile;
+    total_tiles += (int64_t)tiles[b] * n_kv;
+    max_tiles = std::max(max_tiles, tiles[b]);
+  }
+  int tpc = (int)std::max<int64_t>(1, (total_tiles + target - 1) / target);
+  for (; tpc < max_tiles; ++tpc) {
+    int64_t ctas = 0;
+    for (int b = 0; b < n_seqs; ++b) ctas += (int64_t)n_kv * ((tiles[b] + tpc - 1) / tpc);
+    if (ctas <= target) break;
+  }
+  tpc = std::max(1, std::min(tpc, std::max(1, max_tiles)));
+  pl->keys_per_chunk = tpc * pl->tile;
+  pl->n_chunks = std::max(1, (pl->bt.max_len + pl->keys_per_chunk - 1) / pl->keys_per_chunk);
+  pl->off_part = kErrWordBytes;
+  const size_t part_bytes = (size_t)n_seqs * n_kv * pl->n_chunks * pl->R_pad * sizeof(float2);
+  pl->off_raw = round_up(pl->off_part + part_bytes, 256);
+  pl->bytes = pl->off_raw + round_up((size_t)n_kv * pl->bt.T * sizeof(float), 256);
+  return KVC_OK;
+}
+
+// --------------------------------------------------------- decode plan
+struct DecodePlan {
+  int chunk_rows = 0, n_chunks = 0;
+  size_t off_tickets = 0, off_part = 0, bytes = 0;
+};
+
+kvc_status plan_decode(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, int max_kv_len, DecodePlan *pl) {
+  if (dt != KVC_F32 && dt != KVC_BF16) return fail(KVC_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+  if (batch < 1) return fail(KVC_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", batch);
+  if (n_h < 1 || n_kv < 1 || n_h % n_kv != 0)
+    return fail(KVC_ERR_INVALID_ARG, "n_h (%d) must be a positive multiple of n_kv (%d)", n_h, n_kv);
+  const int G = n_h / n_kv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVC_ERR_UNSUPPORTED, "GQA group %d not in {1,2,4,8}", G);
+  if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
+  if (max_kv_len < 0) return fail(KVC_ERR_INVALID_ARG, "max_kv_len must be >= 0");
+  const int64_t units = (int64_t)batch * n_kv;
+  const int64_t want = std::max<int64_t>(1, (4 * kvc::kNumSMs + units - 1) / units);
+  int64_t rows = (max_kv_len + want - 1) / want;
+  rows = std::max<int64_t>(64, (rows + 31) / 32 * 32);
+  pl->chunk_rows = (int)rows;
+  pl->n_chunks = std::max(1, (int)((max_kv_len + rows - 1) / rows));
+  pl->off_tickets = kErrWordBytes;
+  pl->off_part = round_up(pl->off_tickets + (size_t)units * sizeof(int), 256);
+  pl->bytes = pl->off_part + (size_t)units * pl->n_chunks * G * (d_h + 2) * sizeof(float);
+  return KVC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvc_version(void) { return 100; }
+
+const char *kvc_status_string(int status) {
+  switch (status) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_INVALID_ARG: return "KVC_ERR_INVALID_ARG";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
+    case KVC_ERR_WORKSPACE: return "KVC_ERR_WORKSPACE";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+    default: return "KVC_ERR_UNKNOWN";
+  }
+}
+
+const char *kvc_last_error(void) { return g_err; }
+
+uint64_t kvc_cache_bytes(int L, int64_t S, int n_kv, int d_h, int b) {
+  if (L < 0 || S < 0 || n_kv < 0 || d_h < 0 || b < 0) return 0;
+  return 2ull * (uint64_t)L * (uint64_t)S * (uint64_t)n_kv * (uint64_t)d_h * (uint64_t)b;
+}
+
+int64_t kvc_budget_offsets(int n_seqs, const int32_t *seqlens_host, int budget, int32_t *cu_budget_host) {
+  if (n_seqs < 0 || (n_seqs > 0 && !seqlens_host) || !cu_budget_host || budget < 0) return -1;
+  int64_t acc = 0;
+  cu_budget_host[0] = 0;
+  for (int b = 0; b < n_seqs; ++b) {
+    if (seqlens_host[b] < 0) return -1;
+    acc += std::min(budget, seqlens_host[b]);
+    if (acc >= INT32_MAX) return -1;
+    cu_budget_host[b + 1] = (int32_t)acc;
+  }
+  return acc;
+}
+
+size_t kvc_score_window_workspace_size(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int n_h, int n_kv,
+                                       int d_h, int w) {
+  ScorePlan pl;
+  if (plan_score(dt, n_seqs, seqlens_host, n_h, n_kv, d_h, w, &pl) != KVC_OK) return 0;
+  return pl.bytes;
+}
+
+kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                            int n_h, int n_kv, int d_h, int w, int pool_k, float scale, const void *q_win,
+                            const void *k, float *scores, float *scores_raw, void *ws, size_t ws_bytes,
+                            kvc_stream_t stream) {
+  ScorePlan pl;
+  kvc_status s = plan_score(dt, n_seqs, seqlens_host, n_h, n_kv, d_h, w, &pl);
+  if (s != KVC_OK) return s;
+  if (pool_k < 1 || pool_k > 31 || pool_k % 2 == 0)
+    return fail(KVC_ERR_INVALID_ARG, "pool_k must be odd and in [1, 31] (got %d)", pool_k);
+  if (!cu_seqlens) return fail(KVC_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (!aligned16(q_win) || !aligned16(k) || !aligned16(scores))
+    return fail(KVC_ERR_INVALID_ARG, "q_win, k and scores must be non-NULL and 16-byte aligned");
+  if (scores_raw && !aligned16(scores_raw)) return fail(KVC_ERR_INVALID_ARG, "scores_raw must be 16-byte aligned");
+  if (!aligned16(ws) || ws_bytes < pl.bytes)
+    return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes at a 16-byte aligned address (got %zu)", pl.bytes,
+                ws_bytes);
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_h);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  kvc::ScoreArgs a;
+  a.dt = dt; a.n_seqs = n_seqs; a.n_h = n_h; a.n_kv = n_kv; a.d_h = d_h; a.w = w; a.scale = scale;
+  a.cu_seqlens = cu_seqlens; a.q_win = q_win; a.k = k;
+  a.part = reinterpret_cast<float2 *>(wsb + pl.off_part);
+  a.raw = scores_raw ? scores_raw : reinterpret_cast<float *>(wsb + pl.off_raw);
+  a.err = reinterpret_cast<int *>(wsb);
+  a.T_total = (int)pl.bt.T;
+  a.n_chunks = pl.n_chunks;
+  a.keys_per_chunk = pl.keys_per_chunk;
+  a.R_pad = pl.R_pad;
+  cudaError_t e = pl.tc ? kvc::score_window_tc(a, st) : kvc::score_window_simt(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "score kernels");
+  e = kvc::pool_prefix(a.raw, scores, cu_seqlens, n_seqs, n_kv, a.T_total, pl.bt.max_len, w, pool_k, st);
+  if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
+  return KVC_OK;
+}
+
+kvc_status kvc_select_topk(int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                           const int32_t *cu_budget, int n_kv, int w, int budget, const float *scores, int32_t *idx,
+                           kvc_stream_t stream) {
+  Batch bt;
+  kvc_status s = check_batch(n_seqs, seqlens_host, 0, &bt);
+  if (s != KVC_OK) return s;
+  if (n_kv < 1) return fail(KVC_ERR_INVALID_ARG, "n_kv must be >= 1");
+  if (w < 1) return fail(KVC_ERR_INVALID_ARG, "w must be >= 1 (got %d)", w);
+  if (budget < w) return fail(KVC_ERR_INVALID_ARG, "budget (%d) must be >= w (%d): the window is always kept", budget, w);
+  if (!cu_seqlens || !cu_budget) return fail(KVC_ERR_INVALID_ARG, "cu_seqlens / cu_budget is NULL");
+  if (!aligned16(scores) || !aligned16(idx))
+    return fail(KVC_ERR_INVALID_ARG, "scores and idx must be non-NULL and 16-byte aligned");
+  int64_t total = 0;
+  for (int b = 0; b < n_seqs; ++b) total += std::min(budget, seqlens_host[b]);
+  cudaError_t e = kvc::select_topk(scores, idx, cu_seqlens, cu_budget, n_seqs, n_kv, (int)bt.T, (int)total, w, budget,
+                                   std::max(bt.max_len, w), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel");
+  return KVC_OK;
+}
+
+kvc_status kvc_gather_kv(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                         const int32_t *cu_budget, int n_kv, int d_h, int budget, const int32_t *idx, const void *k,
+                         const void *v, void *k_out, void *v_out, kvc_stream_t stream) {
+  const int es = elem_size(dt);
+  if (!es) return fail(KVC_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+  Batch bt;
+  kvc_status s = check_batch(n_seqs, seqlens_host, 0, &bt);
+  if (s != KVC_OK) return s;
+  if (n_kv < 1 || d_h < 1) return fail(KVC_ERR_INVALID_ARG, "n_kv and d_h must be >= 1");
+  if ((d_h * es) % 16 != 0) return fail(KVC_ERR_UNSUPPORTED, "d_h * element size must be a multiple of 16 bytes");
+  if (budget < 0) return fail(KVC_ERR_INVALID_ARG, "budget must be >= 0");
+  if (!cu_seqlens || !cu_budget) return fail(KVC_ERR_INVALID_ARG, "cu_seqlens / cu_budget is NULL");
+  if (!aligned16(idx) || !aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out))
+    return fail(KVC_ERR_INVALID_ARG, "idx, k, v, k_out and v_out must be non-NULL and 16-byte aligned");
+  int64_t total = 0;
+  int max_kept = 0;
+  for (int b = 0; b < n_seqs; ++b) {
+    const int kept = std::min(budget, seqlens_host[b]);
+    total += kept;
+    max_kept = std::max(max_kept, kept);
+  }
+  if (total == 0) return KVC_OK;
+  cudaError_t e = kvc::gather_rows_kv(k, v, k_out, v_out, idx, cu_seqlens, cu_budget, n_seqs, n_kv, d_h * es,
+                                      (int)total, max_kept, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather kernel");
+  return KVC_OK;
+}
+
+size_t kvc_tsp_workspace_size(int S, int w) {
+  if (S < 1 || w < 1 || w > S) return 0;
+  return kErrWordBytes + round_up((size_t)(S - w) * sizeof(float), 256);
+}
+
+kvc_status kvc_tsp_select_gather(kvc_dtype dt, int S, int n_rows, int w, int pool_k, int k_tsp,
+                                 const float *scores_raw, const void *hidden, int D, int32_t *idx_out,
+                                 void *hidden_out, void *ws, size_t ws_bytes, kvc_stream_t stream) {
+  const int es = elem_size(dt);
+  if (!es) return fail(KVC_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+  if (S < 1 || w < 1 || w > S) return fail(KVC_ERR_INVALID_ARG, "need 1 <= w <= S (w=%d, S=%d)", w, S);
+  if (n_rows < 1) return fail(KVC_ERR_INVALID_ARG, "n_rows must be >= 1");
+  if (pool_k < 1 || pool_k > 31 || pool_k % 2 == 0)
+    return fail(KVC_ERR_INVALID_ARG, "pool_k must be odd and in [1, 31] (got %d)", pool_k);
+  if (k_tsp < 0 || k_tsp > S - w) return fail(KVC_ERR_INVALID_ARG, "k_tsp must lie in [0, S - w] (got %d)", k_tsp);
+  if (D < 1 || ((int64_t)D * es) % 16 != 0)
+    return fail(KVC_ERR_UNSUPPORTED, "D * element size must be a positive multiple of 16 bytes");
+  if (!aligned16(scores_raw) || !aligned16(hidden) || !aligned16(idx_out) || !aligned16(hidden_out))
+    return fail(KVC_ERR_INVALID_ARG, "scores_raw, hidden, idx_out and hidden_out must be 16-byte aligned");
+  const size_t need = kvc_tsp_workspace_size(S, w);
+  if (!aligned16(ws) || ws_bytes < need)
+    return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, ws_bytes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float *pooled = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kErrWordBytes);
+  cudaError_t e = kvc::tsp_pool(scores_raw, n_rows, S, w, pool_k, pooled, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tsp pool kernel");
+  e = kvc::tsp_select(pooled, S, w, k_tsp, idx_out, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tsp select kernel");
+  e = kvc::gather_hidden(hidden, hidden_out, idx_out, k_tsp + w, D * es, S, st);
+  if (e != cudaSuccess) return cuda_fail(e, "hidden gather kernel");
+  return KVC_OK;
+}
+
+size_t kvc_gqa_decode_workspace_size(int batch, int n_h, int n_kv, int d_h, int max_kv_len) {
+  DecodePlan pl;
+  if (plan_decode(KVC_BF16, batch, n_h, n_kv, d_h, max_kv_len, &pl) != KVC_OK) return 0;
+  return pl.bytes;
+}
+
+kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, float scale, const void *q,
+                               const void *k_c, const void *v_c, const int64_t *kv_row_offset,
+                               const int32_t *kv_len, int max_kv_len, float *out, void *ws, size_t ws_bytes,
+                               kvc_stream_t stream) {
+  DecodePlan pl;
+  kvc_status s = plan_decode(dt, batch, n_h, n_kv, d_h, max_kv_len, &pl);
+  if (s != KVC_OK) return s;
+  if (!aligned16(q) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(out))
+    return fail(KVC_ERR_INVALID_ARG, "q, k_c, v_c and out must be non-NULL and 16-byte aligned");
+  if (!kv_row_offset || !kv_len) return fail(KVC_ERR_INVALID_ARG, "kv_row_offset / kv_len is NULL");
+  if (!aligned16(ws) || ws_bytes < pl.bytes)
+    return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", pl.bytes, ws_bytes);
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_h);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  kvc::DecodeArgs a;
+  a.dt = dt; a.batch = batch; a.n_h = n_h; a.n_kv = n_kv; a.d_h = d_h; a.scale = scale;
+  a.q = q; a.k_c = k_c; a.v_c = v_c; a.row_off = kv_row_offset; a.kv_len = kv_len; a.out = out;
+  a.tickets = reinterpret_cast<int *>(wsb + pl.off_tickets);
+  a.part = reinterpret_cast<float *>(wsb + pl.off_part);
+  a.n_chunks = pl.n_chunks;
+  a.chunk_rows = pl.chunk_rows;
+  cudaError_t e = kvc::gqa_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
+  return KVC_OK;
+}
+
+}  // extern "C"

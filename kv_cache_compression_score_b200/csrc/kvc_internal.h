@@ -1,0 +1,66 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvc.h"
+
+namespace kvc {
+
+// B200: 148 SMs.  Work plans (and therefore workspace sizes) are computed for
+// this count so that a size query needs no device call.
+constexpr int kNumSMs = 148;
+
+struct ScoreArgs {
+  kvc_dtype dt;
+  int n_seqs, n_h, n_kv, d_h, w;
+  float scale;
+  const int32_t *cu_seqlens;
+  const void *q_win;
+  const void *k;
+  float2 *part;          // [n_seqs, n_kv, n_chunks, R_pad] (m, l) per window row
+  float *raw;            // [n_kv, T_total]
+  int *err;              // device error word (nonzero: a bounded wait gave up)
+  int T_total;
+  int n_chunks;          // key chunks per (sequence, KV head) in the launch grid
+  int keys_per_chunk;    // multiple of the kernel's key tile
+  int R_pad;             // padded window-block rows used for the partials
+};
+
+cudaError_t score_window_simt(const ScoreArgs &a, cudaStream_t st);
+cudaError_t score_window_tc(const ScoreArgs &a, cudaStream_t st);
+int simt_keys_per_tile();
+int tc_keys_per_tile();
+
+cudaError_t pool_prefix(const float *raw, float *scores, const int32_t *cu_seqlens, int n_seqs, int n_kv,
+                        int T_total, int max_len, int w, int pool_k, cudaStream_t st);
+
+cudaError_t select_topk(const float *scores, int32_t *idx, const int32_t *cu_seqlens, const int32_t *cu_budget,
+                        int n_seqs, int n_kv, int T_total, int total_budget, int w, int budget, int max_len,
+                        cudaStream_t st);
+
+cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_out, const int32_t *idx,
+                           const int32_t *cu_seqlens, const int32_t *cu_budget, int n_seqs, int n_kv,
+                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st);
+
+cudaError_t tsp_pool(const float *raw, int n_rows, int S, int w, int pool_k, float *pooled, cudaStream_t st);
+cudaError_t tsp_select(const float *pooled, int S, int w, int k_tsp, int32_t *idx_out, cudaStream_t st);
+cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int n_rows, int row_bytes, int n_src,
+                          cudaStream_t st);
+
+struct DecodeArgs {
+  kvc_dtype dt;
+  int batch, n_h, n_kv, d_h;
+  float scale;
+  const void *q, *k_c, *v_c;
+  const int64_t *row_off;
+  const int32_t *kv_len;
+  float *out;
+  float *part;
+  int *tickets;
+  int n_chunks, chunk_rows;
+};
+cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
+
+}  // namespace kvc

@@ -174,3 +174,16 @@ def packed_batch(seed: int, lengths, n_h: int, n_kv: int, d_h: int, w: int, dtyp
         "cu_seqlens": cu,
         "seqlens": lengths,
     }
+
+
+def index_lists(seed: int, lengths, n_kv: int, budget: int) -> np.ndarray:
+    """Seeded stand-in index lists for gather tests: per (sequence, head) a
+    sorted sample without replacement of min(budget, len) positions of
+    [0, len), concatenated per head -> int32 [n_kv, sum_b min(budget, len_b)]."""
+    rows = [[] for _ in range(n_kv)]
+    for b, L in enumerate(lengths):
+        kept = min(int(budget), int(L))
+        for h in range(n_kv):
+            keys = uniform_u64(stream_key(seed, T_SCORES, b * 256 + h + 1), int(L))
+            rows[h].append(np.sort(np.argsort(keys, kind="stable")[:kept]))
+    return np.stack([np.concatenate(r) if r else np.zeros(0, np.int64) for r in rows]).astype(np.int32)

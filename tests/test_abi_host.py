@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, every
+entry point declared in include/kvc.h is exported and bound, the host helpers
+compute what the pages fix, and invalid arguments are rejected before any
+CUDA call."""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+
+from kv_cache_compression_score_b200 import build as kbuild
+from kv_cache_compression_score_b200 import kvc
+from oracle import kvc_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvc.h")
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kvc.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvc_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in kvc.SIGNATURES, f"{n} has no binding"
+    assert set(kvc.SIGNATURES) == set(names)
+
+
+def test_version_and_status_strings(L):
+    assert kvc.kvc_version() >= 100
+    assert L.kvc_status_string(0) == b"KVC_OK"
+    assert L.kvc_status_string(3) == b"KVC_ERR_WORKSPACE"
+
+
+def test_cache_bytes_matches_worked_example(L):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "cache_bytes.json")))
+    for c in g["cases"]:
+        assert c.get("n_seqs", 1) * kvc.kvc_cache_bytes(c["L"], c["S"], c["n_kv"], c["d_h"], c["b"]) == c["bytes"]
+    assert kvc.kvc_cache_bytes(-1, 4, 1, 1, 1) == 0
+
+
+def test_budget_offsets(L):
+    lens = [100, 3, 50, 0, 7]
+    np.testing.assert_array_equal(kvc.kvc_budget_offsets(lens, 20), O.budget_offsets(lens, 20))
+    with pytest.raises(kvc.KvcError):
+        kvc.kvc_budget_offsets([5, -1], 3)
+
+
+def test_workspace_sizes(L):
+    sl = np.array([32768], dtype=np.int32)
+    n = kvc.kvc_score_window_workspace_size(kvc.KVC_BF16, sl, 32, 8, 128, 32)
+    assert n >= 8 * 32768 * 4                                   # holds the raw scores
+    assert kvc.kvc_score_window_workspace_size(kvc.KVC_BF16, sl, 32, 8, 96, 32) == 0   # d_h unsupported
+    assert kvc.kvc_score_window_workspace_size(kvc.KVC_BF16, np.array([16], np.int32), 32, 8, 128, 32) == 0
+    assert kvc.kvc_tsp_workspace_size(32768, 32) >= (32768 - 32) * 4
+    assert kvc.kvc_tsp_workspace_size(10, 11) == 0
+    assert kvc.kvc_gqa_decode_workspace_size(16, 32, 8, 128, 2048) > 0
+    assert kvc.kvc_gqa_decode_workspace_size(16, 24, 8, 128, 2048) == 0   # G = 3
+
+
+P16 = ctypes.c_void_p(1 << 20)     # aligned fake device address (never dereferenced: calls fail first)
+P8 = ctypes.c_void_p((1 << 20) + 8)
+
+
+def _score(L, **kw):
+    a = dict(dt=kvc.KVC_BF16, n_seqs=1, sl=np.array([64], np.int32), cu=P16, n_h=4, n_kv=2, d_h=128, w=8,
+             pool_k=7, scale=0.0, q=P16, k=P16, sc=P16, raw=None, ws=P16, ws_bytes=1 << 30)
+    a.update(kw)
+    return L.kvc_score_window(a["dt"], a["n_seqs"], a["sl"].ctypes.data_as(ctypes.c_void_p), a["cu"], a["n_h"],
+                              a["n_kv"], a["d_h"], a["w"], a["pool_k"], a["scale"], a["q"], a["k"], a["sc"],
+                              a["raw"], a["ws"], a["ws_bytes"], None)
+
+
+def test_score_window_rejects_before_launch(L):
+    assert _score(L, pool_k=4) == INVALID
+    assert _score(L, pool_k=33) == INVALID
+    assert _score(L, d_h=96) == UNSUPPORTED
+    assert _score(L, dt=7) == UNSUPPORTED
+    assert _score(L, n_h=6, n_kv=4) == INVALID
+    assert _score(L, w=65) == INVALID                     # sequence shorter than the window
+    assert _score(L, n_h=16, n_kv=1, w=32) == UNSUPPORTED  # 512-row window block
+    assert _score(L, q=None) == INVALID
+    assert _score(L, k=P8) == INVALID
+    assert _score(L, raw=P8) == INVALID
+    assert _score(L, ws_bytes=16) == WORKSPACE
+    assert _score(L, n_seqs=0) == INVALID
+
+
+def test_select_gather_decode_tsp_reject_before_launch(L):
+    sl = np.array([100, 40], np.int32)
+    slp = sl.ctypes.data_as(ctypes.c_void_p)
+    # budget below the window
+    assert L.kvc_select_topk(2, slp, P16, P16, 8, 32, 31, P16, P16, None) == INVALID
+    assert b"window" in L.kvc_last_error()
+    assert L.kvc_select_topk(2, slp, None, P16, 8, 32, 64, P16, P16, None) == INVALID
+    assert L.kvc_select_topk(2, slp, P16, P16, 8, 32, 64, P8, P16, None) == INVALID
+    # gather: row bytes must be a multiple of 16
+    assert L.kvc_gather_kv(kvc.KVC_BF16, 2, slp, P16, P16, 8, 4, 64, P16, P16, P16, P16, P16, None) == UNSUPPORTED
+    assert L.kvc_gather_kv(kvc.KVC_BF16, 2, slp, P16, P16, 8, 128, 64, P16, P16, P8, P16, P16, None) == INVALID
+    # decode: group of 3, odd head dim, small workspace
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 24, 8, 128, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 1 << 30,
+                                 None) == UNSUPPORTED
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 80, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 1 << 30,
+                                 None) == UNSUPPORTED
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 128, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 8,
+                                 None) == WORKSPACE
+    # TSP: k_tsp beyond the prefix, even pool
+    assert L.kvc_tsp_select_gather(kvc.KVC_BF16, 100, 8, 32, 7, 69, P16, P16, 4096, P16, P16, P16, 1 << 20,
+                                   None) == INVALID
+    assert L.kvc_tsp_select_gather(kvc.KVC_BF16, 100, 8, 32, 6, 10, P16, P16, 4096, P16, P16, P16, 1 << 20,
+                                   None) == INVALID
+    assert L.kvc_tsp_select_gather(kvc.KVC_BF16, 100, 8, 32, 7, 10, P16, P16, 4, P16, P16, P16, 1 << 20,
+                                   None) == UNSUPPORTED
