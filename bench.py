@@ -1,0 +1,379 @@
+"""Benchmark of the observation-window KV-compression hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+
+One step = one pass of the whole path over one batch of seeded synthetic input
+(Llama-3-8B-shaped layer: n_h 32, n_kv 8, d_h 128, bf16, S 32768, window 32,
+pool 7, budget 2048, 1% of keys boosted):
+  kvc_score_window -> kvc_select_topk -> kvc_gather_kv for one sequence, then
+  kvc_gqa_decode_attn for a batch of 16 compact caches (cache 0 is the one the
+  step's gather writes; caches 1..15 are seeded stand-ins of the same shape).
+
+value = K tokens/s of score + select + gather (S / time / 1e3), whole job over
+all ranks; decode GB/s and the per-call breakdown are extra keys.  Timing: CUDA
+events around every step on the launching stream, L2 flushed (256 MiB write)
+between steps outside the events, max over ranks.  With N > 1 every rank runs
+its own sequences (weak scaling, no collective on the data path).
+
+--impl reference runs the fp64 CPU oracle on the same workload and metric
+(rank 0 only; the pages ship no code, so the oracle is the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CONFIG2 = dict(name="llama3-8b-layer-S32768-B2048", n_h=32, n_kv=8, d_h=128, S=32768, w=32, pool_k=7, budget=2048,
+               decode_batch=16, boost_frac=0.01, boost=3.0, seed=1002, dtype="bf16")
+METRIC = "score+select+gather K-tok/s & GB/s at S=32K; decode-attn GB/s vs 8 TB/s HBM"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def env_rank():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(cfg):
+    """Bytes the path must move: K read once by scoring; retained K/V rows read
+    and written by the gather; every retained K/V row read by decode."""
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    row = cfg["n_kv"] * cfg["d_h"] * esz
+    score = cfg["S"] * row
+    gather = 2 * 2 * cfg["budget"] * row
+    decode = 2 * cfg["decode_batch"] * cfg["budget"] * row
+    return score, gather, decode
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9 and parts[1].isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [int(r[1]) for r in rows]
+        mx = int(rows[0][2])
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": int(statistics.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, local_rank, world = env_rank()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+
+    from kv_cache_compression_score_b200 import build as kbuild
+    if rank == 0 or world == 1:
+        kbuild.build()
+    if world > 1:
+        dist.barrier()
+    from kv_cache_compression_score_b200 import synth
+    from kv_cache_compression_score_b200.runner import Compressor, Decoder, to_device
+
+    cfg = dict(CONFIG2)
+    seed = cfg["seed"] + 100 * rank
+    S, n_h, n_kv, d, w, B, nb = cfg["S"], cfg["n_h"], cfg["n_kv"], cfg["d_h"], cfg["w"], cfg["budget"], \
+        cfg["decode_batch"]
+    bt = synth.packed_batch(seed, [S], n_h, n_kv, d, w, cfg["dtype"], cfg["boost_frac"], cfg["boost"])
+    q_win, k, v = (to_device(bt[x], cfg["dtype"], dev) for x in ("q_win", "k", "v"))
+    comp = Compressor(cfg["dtype"], [S], n_h, n_kv, d, w, cfg["pool_k"], B, device=dev, keep_raw=False)
+    # 16 compact caches in one buffer; slot 0 is written by the step's gather
+    kc_all = torch.empty((nb * B, n_kv, d), dtype=torch.bfloat16, device=dev)
+    vc_all = torch.empty_like(kc_all)
+    for b in range(1, nb):
+        kk, vv = synth.keys_values(seed + 7, b, B, n_kv, d, cfg["dtype"])
+        kc_all[b * B:(b + 1) * B].copy_(to_device(kk, cfg["dtype"], dev))
+        vc_all[b * B:(b + 1) * B].copy_(to_device(vv, cfg["dtype"], dev))
+    comp.buf.k_c = kc_all[:B]
+    comp.buf.v_c = vc_all[:B]
+    qd = to_device(synth.decode_queries(seed + 8, nb, n_h, d, cfg["dtype"]), cfg["dtype"], dev)
+    off = torch.arange(nb, dtype=torch.int64, device=dev) * B
+    ln = torch.full((nb,), B, dtype=torch.int32, device=dev)
+    dec = Decoder(nb, n_h, n_kv, d, B, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)    # 256 MiB > 2x L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs: evs[0].record(stream)
+        comp.score(q_win, k, stream)
+        if evs: evs[1].record(stream)
+        comp.select(stream)
+        if evs: evs[2].record(stream)
+        comp.gather(k, v, stream)
+        if evs: evs[3].record(stream)
+        dec.run(qd, kc_all, vc_all, off, ln, stream)
+        if evs: evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert comp.device_error_word() == 0, "device error word set"
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])  # ms
+    mean = per.mean(axis=0)
+    t_ssg = float(mean[:3].sum())
+    t_step = float(mean.sum())
+    t_dec = float(mean[3])
+    if world > 1:
+        tt = torch.tensor([t_ssg, t_step, t_dec], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_ssg, t_step, t_dec = tt.tolist()
+
+    # ---- e2e: the same path through the C ABI with pinned host buffers
+    e2e = run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush)
+    if world > 1:
+        tt = torch.tensor([e2e["t_ms"]], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e["t_ms"] = float(tt.item())
+
+    score_b, gather_b, decode_b = algorithmic_bytes(cfg)
+    hbm, peak_kind = measured_peaks()
+    ssg_gbs = (score_b + gather_b) / (t_ssg * 1e-3) / 1e9
+    dec_gbs = decode_b / (t_dec * 1e-3) / 1e9
+    # dominant call by time -> roofline object (all HBM-bound)
+    calls = {"score": (mean[0], score_b), "select": (mean[1], 0), "gather": (mean[2], gather_b),
+             "decode": (mean[3], decode_b)}
+    dom = max(calls, key=lambda c: calls[c][0])
+    dom_gbs = calls[dom][1] / (calls[dom][0] * 1e-3) / 1e9 if calls[dom][1] else 0.0
+    traffic = load_traffic(dom)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(world * S / (t_ssg * 1e-3) / 1e3, 1),
+            "unit": "K-tok/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t_step, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": cfg["dtype"],
+            "data": "synthetic (seeded N(0,1), 1% keys boosted +3 sigma)",
+            "config": {"workload": cfg["name"], "n_h": n_h, "n_kv": n_kv, "d_h": d, "seq_len": S, "window": w,
+                       "pool": cfg["pool_k"], "budget": B, "decode_batch": nb,
+                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "parallelism": f"replicas x{world}"},
+            "gbs": round(ssg_gbs, 1),
+            "decode": {"gbs": round(dec_gbs, 1), "us": round(t_dec * 1e3, 2), "frac_of_8000": round(dec_gbs / 8000, 3)},
+            "breakdown_us": {c: round(float(calls[c][0]) * 1e3, 2) for c in calls},
+            "ssg_us": round(t_ssg * 1e3, 2),
+            "ssg_frac_of_8000": round(ssg_gbs / 8000, 3),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": hbm,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / hbm, 3),
+                         "traffic": traffic},
+            "e2e": {"value": round(world * S / (e2e["t_ms"] * 1e-3) / 1e3, 2), "unit": "K-tok/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clocks,
+            "wall_s_timed_region": round(t_wall, 3),
+        }
+        line["cpu_baseline"] = cpu_baseline(cfg, bt) if world == 1 else None
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush):
+    """Inputs copied host->device from pinned memory and results device->host
+    inside the timed region, every step."""
+    import torch
+    from kv_cache_compression_score_b200.runner import to_device
+
+    h_q = to_device(bt["q_win"], cfg["dtype"], "cpu").pin_memory()
+    h_k = to_device(bt["k"], cfg["dtype"], "cpu").pin_memory()
+    h_v = to_device(bt["v"], cfg["dtype"], "cpu").pin_memory()
+    h_qd = qd.cpu().pin_memory()
+    d_q, d_k, d_v = torch.empty_like(h_q, device=dev), torch.empty_like(h_k, device=dev), torch.empty_like(h_v, device=dev)
+    h_idx = torch.empty(comp.buf.idx.shape, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(dec.out.shape, dtype=torch.float32).pin_memory()
+    n = max(3, min(args.steps, 10))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n + 1)]
+    for i in range(n + 1):             # first iteration untimed (warm-up)
+        flush.zero_()
+        evs[i][0].record(stream)
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        qd.copy_(h_qd, non_blocking=True)
+        comp.score(d_q, d_k, stream)
+        comp.select(stream)
+        comp.gather(d_k, d_v, stream)
+        dec.run(qd, kc_all, vc_all, off, ln, stream)
+        h_idx.copy_(comp.buf.idx, non_blocking=True)
+        h_out.copy_(dec.out, non_blocking=True)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    t = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(1, n + 1))
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_k, h_v, h_qd))
+    d2h = h_idx.numel() * 4 + h_out.numel() * 4
+    return {"t_ms": t, "h2d": h2d, "d2h": d2h}
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of the dominant call from the committed ncu summary, if current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("current", False):
+            return e.get("bytes_per_launch")
+    return None
+
+
+# ----------------------------------------------------------- oracle arm
+def oracle_step(cfg, bt):
+    from oracle import kvc_oracle as O
+    cu = bt["cu_seqlens"]
+    raw = O.raw_scores(bt["q_win"], bt["k"], cu, cfg["n_h"], cfg["n_kv"], cfg["w"], cfg["dtype"])
+    pooled = O.pool_prefix(raw, cu, cfg["w"], cfg["pool_k"])
+    idx = O.select_topk(pooled, cu, cfg["w"], cfg["budget"])
+    O.gather_kv(bt["k"], bt["v"], idx, cu, cfg["budget"])
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, bt, budget_s=10.0):
+    """The oracle, as it stands, on one full layer of the same workload
+    (score + select + gather over all KV heads), repeated for ~10 s."""
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(cfg, bt)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    t = time.perf_counter() - t0
+    return {"value": round(reps * cfg["S"] / t / 1e3, 3), "unit": "K-tok/s", "cores": oracle_threads(),
+            "kind": "oracle", "sample": f"{reps} full layers (S={cfg['S']}, all {cfg['n_kv']} KV heads) in {t:.1f} s"}
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return
+    from kv_cache_compression_score_b200 import synth
+    cfg = dict(CONFIG2)
+    bt = synth.packed_batch(cfg["seed"], [cfg["S"]], cfg["n_h"], cfg["n_kv"], cfg["d_h"], cfg["w"], cfg["dtype"],
+                            cfg["boost_frac"], cfg["boost"])
+    for _ in range(args.warmup):
+        oracle_step(cfg, bt)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(cfg, bt)
+        ts.append(time.perf_counter() - t0)
+    t = statistics.mean(ts)
+    v = round(world * cfg["S"] / t / 1e3, 3)
+    line = {"metric": METRIC, "value": v, "unit": "K-tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), 1% keys boosted +3 sigma)",
+            "config": {"workload": cfg["name"], "n_h": cfg["n_h"], "n_kv": cfg["n_kv"], "d_h": cfg["d_h"],
+                       "seq_len": cfg["S"], "window": cfg["w"], "pool": cfg["pool_k"], "budget": cfg["budget"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "K-tok/s", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": f"one full layer per step (S={cfg['S']}, all KV heads), score+select+gather"},
+            "e2e": {"value": v, "unit": "K-tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

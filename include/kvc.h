@@ -180,7 +180,8 @@ kvc_status kvc_tsp_select_gather(kvc_dtype dt, int S, int n_rows, int w, int poo
  *                   * Vc[o_b + t][h],   h = qh / G,  o_b = kv_row_offset[b]
  * and 0 when kv_len[b] == 0.  Offsets may alias (several queries on one cache).
  *
- * q: [batch, n_h, d_h] of dt;  k_c, v_c: [rows, n_kv, d_h] of dt;
+ * q: [batch, n_h, d_h] of dt;  k_c, v_c: [cache_rows, n_kv, d_h] of dt, with
+ * kv_row_offset[b] + kv_len[b] <= cache_rows (cache_rows < 2^31);
  * kv_row_offset: device int64[batch];  kv_len: device int32[batch], each
  * <= max_kv_len;  out: float32 [batch, n_h, d_h].  G in {1, 2, 4, 8};
  * d_h in {64, 128}.  ws: kvc_gqa_decode_workspace_size() bytes, counters
@@ -188,7 +189,7 @@ kvc_status kvc_tsp_select_gather(kvc_dtype dt, int S, int n_rows, int w, int poo
  * ------------------------------------------------------------------------ */
 size_t kvc_gqa_decode_workspace_size(int batch, int n_h, int n_kv, int d_h, int max_kv_len);
 kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, float scale,
-                               const void *q, const void *k_c, const void *v_c,
+                               const void *q, const void *k_c, const void *v_c, int64_t cache_rows,
                                const int64_t *kv_row_offset, const int32_t *kv_len,
                                int max_kv_len, float *out, void *ws, size_t ws_bytes,
                                kvc_stream_t stream);

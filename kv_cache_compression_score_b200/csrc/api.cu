@@ -125,10 +125,13 @@ kvc_status plan_decode(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, int 
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVC_ERR_UNSUPPORTED, "GQA group %d not in {1,2,4,8}", G);
   if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
   if (max_kv_len < 0) return fail(KVC_ERR_INVALID_ARG, "max_kv_len must be >= 0");
+  // chunks of whole tiles such that the persistent grid (2 CTAs per SM) gets
+  // about six work items per CTA
   const int64_t units = (int64_t)batch * n_kv;
-  const int64_t want = std::max<int64_t>(1, (4 * kvc::kNumSMs + units - 1) / units);
-  int64_t rows = (max_kv_len + want - 1) / want;
-  rows = std::max<int64_t>(64, (rows + 31) / 32 * 32);
+  const int tile = kvc::decode_tile_rows();
+  const int64_t target_items = 6 * 2 * kvc::kNumSMs;
+  int64_t rows = (int64_t)max_kv_len * units / target_items;
+  rows = std::max<int64_t>(2 * tile, (rows + tile - 1) / tile * tile);
   pl->chunk_rows = (int)rows;
   pl->n_chunks = std::max(1, (int)((max_kv_len + rows - 1) / rows));
   pl->off_tickets = kErrWordBytes;
@@ -305,7 +308,7 @@ size_t kvc_gqa_decode_workspace_size(int batch, int n_h, int n_kv, int d_h, int 
 }
 
 kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, float scale, const void *q,
-                               const void *k_c, const void *v_c, const int64_t *kv_row_offset,
+                               const void *k_c, const void *v_c, int64_t cache_rows, const int64_t *kv_row_offset,
                                const int32_t *kv_len, int max_kv_len, float *out, void *ws, size_t ws_bytes,
                                kvc_stream_t stream) {
   DecodePlan pl;
@@ -314,6 +317,8 @@ kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d
   if (!aligned16(q) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(out))
     return fail(KVC_ERR_INVALID_ARG, "q, k_c, v_c and out must be non-NULL and 16-byte aligned");
   if (!kv_row_offset || !kv_len) return fail(KVC_ERR_INVALID_ARG, "kv_row_offset / kv_len is NULL");
+  if (cache_rows < 1 || cache_rows > INT32_MAX)
+    return fail(KVC_ERR_INVALID_ARG, "cache_rows must lie in [1, 2^31) (got %lld)", (long long)cache_rows);
   if (!aligned16(ws) || ws_bytes < pl.bytes)
     return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", pl.bytes, ws_bytes);
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_h);
@@ -322,6 +327,8 @@ kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d
   a.dt = dt; a.batch = batch; a.n_h = n_h; a.n_kv = n_kv; a.d_h = d_h; a.scale = scale;
   a.q = q; a.k_c = k_c; a.v_c = v_c; a.row_off = kv_row_offset; a.kv_len = kv_len; a.out = out;
   a.tickets = reinterpret_cast<int *>(wsb + pl.off_tickets);
+  a.err = reinterpret_cast<int *>(wsb);
+  a.cache_rows = cache_rows;
   a.part = reinterpret_cast<float *>(wsb + pl.off_part);
   a.n_chunks = pl.n_chunks;
   a.chunk_rows = pl.chunk_rows;

@@ -1,0 +1,120 @@
+// Compact-cache gather (SnapKV keeps the chosen subset of past keys and
+// values, "Variantes de l'attention et compression du cache KV", section
+// "Compresser un cache existant") and hidden-state gather (FastKV token-
+// selective propagation, FastKV section 2.A).  Both are HBM streams of
+// 16-byte vector loads and stores; an index outside its sequence yields a
+// zero row instead of an out-of-bounds read.
+#include "kvc_common.cuh"
+#include "kvc_internal.h"
+
+namespace kvc {
+namespace {
+
+// ------------------------------------------------------------------- gathers
+constexpr int kGatherThreads = 256;
+constexpr int kGatherUnroll = 4;
+
+// One 16-byte vector of one (slot t, head h) row per work item.
+__global__ void __launch_bounds__(kGatherThreads)
+gather_kv_kernel(const uint8_t *__restrict__ k, const uint8_t *__restrict__ v, uint8_t *__restrict__ k_out,
+                 uint8_t *__restrict__ v_out, const int32_t *__restrict__ idx, const int *__restrict__ cu_seqlens,
+                 const int *__restrict__ cu_budget, int n_kv, int vec_per_head, int total_budget) {
+  const int b = blockIdx.y;
+  const int t0 = cu_seqlens[b], len = cu_seqlens[b + 1] - t0;
+  const int cb = cu_budget[b], kept = cu_budget[b + 1] - cb;
+  const int row_vecs = n_kv * vec_per_head;
+  const long long n_items = (long long)kept * row_vecs;
+  const size_t head_bytes = (size_t)vec_per_head * 16;
+  for (long long base = (long long)blockIdx.x * kGatherThreads * kGatherUnroll + threadIdx.x; base < n_items;
+       base += (long long)gridDim.x * kGatherThreads * kGatherUnroll) {
+    uint4 kv_k[kGatherUnroll], kv_v[kGatherUnroll];
+    size_t dst_off[kGatherUnroll];
+    bool ok[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const long long e = base + (long long)u * kGatherThreads;
+      ok[u] = e < n_items;
+      if (ok[u]) {
+        const int t = (int)(e / row_vecs);
+        const int rem = (int)(e - (long long)t * row_vecs);
+        const int h = rem / vec_per_head, c = rem - h * vec_per_head;
+        const int src_t = idx[(size_t)h * total_budget + cb + t];
+        dst_off[u] = ((size_t)(cb + t) * n_kv + h) * head_bytes + (size_t)c * 16;
+        if (src_t >= 0 && src_t < len) {
+          const size_t src_off = ((size_t)(t0 + src_t) * n_kv + h) * head_bytes + (size_t)c * 16;
+          kv_k[u] = ld_stream16(k + src_off);
+          kv_v[u] = ld_stream16(v + src_off);
+        } else {   // index outside the sequence: zero row, no out-of-bounds read
+          kv_k[u] = make_uint4(0, 0, 0, 0);
+          kv_v[u] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      if (ok[u]) {
+        st_stream16(k_out + dst_off[u], kv_k[u]);
+        st_stream16(v_out + dst_off[u], kv_v[u]);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kGatherThreads)
+gather_hidden_kernel(const uint8_t *__restrict__ hidden, uint8_t *__restrict__ out, const int32_t *__restrict__ idx,
+                     int n_rows, int vec_per_row, int n_src) {
+  const long long n_items = (long long)n_rows * vec_per_row;
+  for (long long base = (long long)blockIdx.x * kGatherThreads * kGatherUnroll + threadIdx.x; base < n_items;
+       base += (long long)gridDim.x * kGatherThreads * kGatherUnroll) {
+    uint4 val[kGatherUnroll];
+    size_t dst_off[kGatherUnroll];
+    bool ok[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const long long e = base + (long long)u * kGatherThreads;
+      ok[u] = e < n_items;
+      if (ok[u]) {
+        const int t = (int)(e / vec_per_row), c = (int)(e - (long long)t * vec_per_row);
+        const size_t row_bytes = (size_t)vec_per_row * 16;
+        dst_off[u] = (size_t)t * row_bytes + (size_t)c * 16;
+        const int src = idx[t];
+        val[u] = (src >= 0 && src < n_src) ? ld_stream16(hidden + (size_t)src * row_bytes + (size_t)c * 16)
+                                           : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u)
+      if (ok[u]) st_stream16(out + dst_off[u], val[u]);
+  }
+}
+
+}  // namespace
+
+cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_out, const int32_t *idx,
+                           const int32_t *cu_seqlens, const int32_t *cu_budget, int n_seqs, int n_kv,
+                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st) {
+  const int vph = row_bytes_per_head / 16;
+  const long long items = (long long)max_kept * n_kv * vph;
+  long long blocks = (items + kGatherThreads * kGatherUnroll - 1) / (kGatherThreads * kGatherUnroll);
+  if (blocks < 1) blocks = 1;
+  if (blocks > 65535) blocks = 65535;
+  dim3 grid((unsigned)blocks, n_seqs);
+  gather_kv_kernel<<<grid, kGatherThreads, 0, st>>>(
+      static_cast<const uint8_t *>(k), static_cast<const uint8_t *>(v), static_cast<uint8_t *>(k_out),
+      static_cast<uint8_t *>(v_out), idx, cu_seqlens, cu_budget, n_kv, vph, total_budget);
+  return cudaGetLastError();
+}
+
+cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int n_rows, int row_bytes, int n_src,
+                          cudaStream_t st) {
+  if (n_rows == 0) return cudaSuccess;
+  const int vpr = row_bytes / 16;
+  const long long items = (long long)n_rows * vpr;
+  long long blocks = (items + kGatherThreads * kGatherUnroll - 1) / (kGatherThreads * kGatherUnroll);
+  if (blocks > 65535) blocks = 65535;
+  gather_hidden_kernel<<<(unsigned)blocks, kGatherThreads, 0, st>>>(
+      static_cast<const uint8_t *>(hidden), static_cast<uint8_t *>(out), idx, n_rows, vpr, n_src);
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -59,8 +59,11 @@ struct DecodeArgs {
   float *out;
   float *part;
   int *tickets;
+  int *err;              // device error word
+  int64_t cache_rows;    // rows of k_c / v_c (tensor-map extent)
   int n_chunks, chunk_rows;
 };
 cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
+int decode_tile_rows();
 
 }  // namespace kvc

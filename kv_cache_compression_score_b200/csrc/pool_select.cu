@@ -81,7 +81,7 @@ tsp_pool_kernel(const float *__restrict__ raw, int n_rows, int S, int w, int r, 
 // ---------------------------------------------------------------- selection
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSmemKeysMax = 40960;   // keys cached in shared memory (160 KB)
+constexpr int kSmemKeysMax = 40960;   // keys cached in shared memory (+1 pad word per 32: 165 KB)
 
 // float -> uint32 with the same order (negatives below positives, NaN on top)
 KVC_DEVINL uint32_t order_key(float f) {
@@ -90,107 +90,147 @@ KVC_DEVINL uint32_t order_key(float f) {
 }
 
 struct SelSmem {
-  int hist[4096];
+  int hist[2048];
   int wsum[kSelWarps];
+  int wsum2[kSelWarps];
   int bcast[4];
 };
 
-// Block-wide exclusive prefix sum of one int per thread; returns the
-// exclusive value and writes the block total to *total.
-KVC_DEVINL int block_exclusive_scan(int v, SelSmem &sm, int *total) {
+// Block-wide exclusive prefix sum of an int2 per thread (two counters at once).
+KVC_DEVINL int2 block_exclusive_scan2(int2 v, SelSmem &sm, int2 *total) {
   const int lane = lane_id(), wid = warp_id();
-  int x = v;
+  int x = v.x, y = v.y;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const int a = __shfl_up_sync(0xffffffffu, x, o), b = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) { x += a; y += b; }
   }
-  if (lane == 31) sm.wsum[wid] = x;
+  if (lane == 31) { sm.wsum[wid] = x; sm.wsum2[wid] = y; }
   __syncthreads();
   if (wid == 0) {
-    int s = sm.wsum[lane];
+    int a = sm.wsum[lane], b = sm.wsum2[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
+      const int c = __shfl_up_sync(0xffffffffu, a, o), d = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) { a += c; b += d; }
     }
-    sm.wsum[lane] = s;   // inclusive warp prefix
+    sm.wsum[lane] = a;
+    sm.wsum2[lane] = b;
   }
   __syncthreads();
-  const int before = (wid == 0) ? 0 : sm.wsum[wid - 1];
-  *total = sm.wsum[kSelWarps - 1];
-  const int ex = before + x - v;
+  const int bx = wid ? sm.wsum[wid - 1] : 0, by = wid ? sm.wsum2[wid - 1] : 0;
+  *total = make_int2(sm.wsum[kSelWarps - 1], sm.wsum2[kSelWarps - 1]);
   __syncthreads();
-  return ex;
+  return make_int2(bx + x - v.x, by + y - v.y);
 }
 
 // Writes the ascending positions of the k largest of src[0..n) (lowest index
 // first among equal keys) to out[0..k).  0 <= k <= n.
+//
+// Thread t owns the contiguous run [t*E, (t+1)*E), E = ceil(n / threads), so
+// index order is (thread, position in run).  Keys are cached in shared memory
+// with one pad word per 32 (conflict-free strided reads) when n fits the
+// cache, else re-read from global memory (L2-resident).  Radix digits of 11
+// bits start at the highest bit where the keys of the array differ, so the
+// first histogram spreads over the occupied range.
 KVC_DEVINL void block_topk_ascending(const float *__restrict__ src, int n, int k, int32_t *__restrict__ out,
                                      uint32_t *cache, int cache_cap, SelSmem &sm) {
   if (k <= 0) return;
-  const bool cached = (n <= cache_cap);
   if (k >= n) {
     for (int i = threadIdx.x; i < n; i += kSelThreads) out[i] = i;
     return;
   }
-  if (cached)
-    for (int i = threadIdx.x; i < n; i += kSelThreads) cache[i] = order_key(src[i]);
-  // cache writes are ordered before the first histogram read by the syncs below
-  uint32_t prefix = 0, pmask = 0;
-  int k_rem = k;
-  const int shifts[3] = {20, 10, 0};
-  const int widths[3] = {12, 10, 10};
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass], nb = 1 << widths[pass];
-    for (int i = threadIdx.x; i < nb; i += kSelThreads) sm.hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += kSelThreads) {
-      const uint32_t u = cached ? cache[i] : order_key(src[i]);
-      if ((u & pmask) == prefix) atomicAdd(&sm.hist[(u >> shift) & (nb - 1)], 1);
-    }
-    __syncthreads();
-    // suffix counts: thread t owns bins [t*per, (t+1)*per) counted from the top
-    const int per = nb / kSelThreads;   // 4 or 1
-    int own = 0;
-    for (int q = 0; q < per; ++q) own += sm.hist[nb - 1 - (threadIdx.x * per + q)];
-    int tot;
-    const int above = block_exclusive_scan(own, sm, &tot);   // keys in higher bins
-    int run = above;
-    for (int q = 0; q < per; ++q) {
-      const int bin = nb - 1 - (threadIdx.x * per + q);
-      const int cnt = sm.hist[bin];
-      if (run < k_rem && run + cnt >= k_rem) {
-        sm.bcast[0] = bin;
-        sm.bcast[1] = run;
-      }
-      run += cnt;
-    }
-    __syncthreads();
-    const int bin = sm.bcast[0];
-    k_rem -= sm.bcast[1];
-    prefix |= (uint32_t)bin << shift;
-    pmask |= (uint32_t)(nb - 1) << shift;
+  const bool cached = (n <= cache_cap);
+  const int E = (n + kSelThreads - 1) / kSelThreads;
+  const int beg = min(n, (int)threadIdx.x * E), end = min(n, beg + E);
+  auto key_at = [&](int i) -> uint32_t { return cached ? cache[i + (i >> 5)] : order_key(src[i]); };
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  if (cached) {
+    for (int i = threadIdx.x; i < n; i += kSelThreads) cache[i + (i >> 5)] = order_key(src[i]);
     __syncthreads();
   }
-  const uint32_t T = prefix;   // key of the k-th largest element; take k_rem of the keys == T
-  int run_gt = 0, run_eq = 0;
-  for (int base = 0; base < n; base += kSelThreads) {
-    const int i = base + threadIdx.x;
-    int gt = 0, eq = 0;
-    if (i < n) {
-      const uint32_t u = cached ? cache[i] : order_key(src[i]);
-      gt = u > T;
-      eq = u == T;
+  for (int i = beg; i < end; ++i) {
+    const uint32_t u = key_at(i);
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  }
+  // block min / max
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane_id() == 0) { sm.wsum[warp_id()] = (int)kmin; sm.wsum2[warp_id()] = (int)kmax; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t a = 0xffffffffu, b = 0u;
+    for (int q = 0; q < kSelWarps; ++q) { a = min(a, (uint32_t)sm.wsum[q]); b = max(b, (uint32_t)sm.wsum2[q]); }
+    sm.bcast[2] = (int)a;
+    sm.bcast[3] = (int)b;
+  }
+  __syncthreads();
+  kmin = (uint32_t)sm.bcast[2];
+  kmax = (uint32_t)sm.bcast[3];
+  __syncthreads();
+
+  uint32_t prefix = kmin, pmask = 0u;        // bits above `top` are common to every key
+  int k_rem = k;
+  if (kmin != kmax) {
+    const int top = 31 - __clz(kmin ^ kmax);  // highest differing bit
+    pmask = (top == 31) ? 0u : (0xffffffffu << (top + 1));
+    prefix = kmin & pmask;
+    for (int hi = top; hi >= 0; hi -= 11) {
+      const int width = min(11, hi + 1), shift = hi + 1 - width, nb = 1 << width;
+      for (int i = threadIdx.x; i < nb; i += kSelThreads) sm.hist[i] = 0;
+      __syncthreads();
+      for (int i = beg; i < end; ++i) {
+        const uint32_t u = key_at(i);
+        if ((u & pmask) == prefix) atomicAdd(&sm.hist[(u >> shift) & (nb - 1)], 1);
+      }
+      __syncthreads();
+      // suffix counts from the top bin down: thread t owns bins nb-1-(t*per + q)
+      const int per = (nb + kSelThreads - 1) / kSelThreads;
+      int own = 0;
+      for (int q = 0; q < per; ++q) {
+        const int bin = nb - 1 - ((int)threadIdx.x * per + q);
+        if (bin >= 0) own += sm.hist[bin];
+      }
+      int2 tot;
+      const int above = block_exclusive_scan2(make_int2(own, 0), sm, &tot).x;
+      int run = above;
+      for (int q = 0; q < per; ++q) {
+        const int bin = nb - 1 - ((int)threadIdx.x * per + q);
+        if (bin < 0) break;
+        const int cnt = sm.hist[bin];
+        if (run < k_rem && run + cnt >= k_rem) { sm.bcast[0] = bin; sm.bcast[1] = run; }
+        run += cnt;
+      }
+      __syncthreads();
+      k_rem -= sm.bcast[1];
+      prefix |= (uint32_t)sm.bcast[0] << shift;
+      pmask |= (uint32_t)(nb - 1) << shift;
+      __syncthreads();
     }
-    int tot;
-    const int ex = block_exclusive_scan(gt | (eq << 16), sm, &tot);
-    const int ex_gt = ex & 0xffff, ex_eq = ex >> 16;
-    const int eq_before = run_eq + ex_eq;
-    if (gt || (eq && eq_before < k_rem)) out[run_gt + ex_gt + min(eq_before, k_rem)] = i;
-    run_gt += tot & 0xffff;
-    run_eq += tot >> 16;
+  }
+  const uint32_t T = prefix;   // key of the k-th largest; take the first k_rem keys equal to T
+  int gt = 0, eq = 0;
+  for (int i = beg; i < end; ++i) {
+    const uint32_t u = key_at(i);
+    gt += u > T;
+    eq += u == T;
+  }
+  int2 tot;
+  const int2 ex = block_exclusive_scan2(make_int2(gt, eq), sm, &tot);
+  int g_before = ex.x, e_before = ex.y;
+  for (int i = beg; i < end; ++i) {
+    const uint32_t u = key_at(i);
+    if (u > T) {
+      out[g_before + min(e_before, k_rem)] = i;
+      ++g_before;
+    } else if (u == T) {
+      if (e_before < k_rem) out[g_before + e_before] = i;
+      ++e_before;
+    }
   }
 }
 
@@ -241,8 +281,9 @@ cudaError_t tsp_pool(const float *raw, int n_rows, int S, int w, int pool_k, flo
 
 static cudaError_t set_sel_smem(const void *fn, int n, int *cap, size_t *bytes) {
   *cap = n <= kSmemKeysMax ? n : 0;
-  *bytes = (size_t)(*cap) * sizeof(uint32_t);
-  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSmemKeysMax * 4));
+  *bytes = (size_t)(*cap + *cap / 32 + 1) * sizeof(uint32_t);
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)((kSmemKeysMax + kSmemKeysMax / 32 + 1) * 4));
 }
 
 cudaError_t select_topk(const float *scores, int32_t *idx, const int32_t *cu_seqlens, const int32_t *cu_budget,

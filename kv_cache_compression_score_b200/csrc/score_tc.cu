@@ -85,6 +85,58 @@ KVC_DEVINL void stage_q(uint8_t *sq, const TcParams &p, int b, int h, int tid, i
 
 KVC_DEVINL void set_err(int *err, int code) { atomicCAS(err, 0, code); }
 
+// Stats-pass reduction of 32 logits of one window row (keys k0..k0+31):
+// online max / sum of 2^(c*z - m), masked keys (beyond the chunk end or the
+// row's causal limit) contribute nothing.
+KVC_DEVINL void epi_stats_chunk(float *v, int k0, int key_end, int P, int row_pos, float c, float &m, float &l) {
+  if (!(k0 + 31 <= P && k0 + 32 <= key_end)) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int key = k0 + j;
+      if (!(key < key_end && key <= row_pos)) v[j] = kNegInf;
+    }
+  }
+  float t[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) t[j] = fmaxf(t[j], t[j + 8]);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) t[j] = fmaxf(t[j], t[j + 4]);
+  const float cmax = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])) * c;   // c > 0
+  const float mn = fmaxf(m, cmax);
+  const float ms = (mn == kNegInf) ? 0.f : mn;
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = fast_exp2(fmaf(v[j], c, -ms));
+#pragma unroll
+  for (int j = 8; j < 32; ++j) a[j & 7] += fast_exp2(fmaf(v[j], c, -ms));
+  const float cs = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  l = fmaf(l, fast_exp2(m - ms), cs);
+  m = mn;
+}
+
+// Score-pass accumulation for one key over window rows r0..r0+31:
+// acc += 2^(c*z_r - off_r), rows above the key's causal limit skipped.
+template <typename Params>
+KVC_DEVINL void epi_score_chunk(const float *v, const float *off, int r0, int key, int P, const Params &p,
+                                float *acc8) {
+  if (key <= P) {     // prefix key (or the first window key): visible to every row
+#pragma unroll
+    for (int r = 0; r < 32; r += 4) {
+      const float4 o4 = *reinterpret_cast<const float4 *>(off + r0 + r);
+      acc8[(r >> 2) & 7] += fast_exp2(fmaf(v[r], p.c, -o4.x)) + fast_exp2(fmaf(v[r + 1], p.c, -o4.y)) +
+                            (fast_exp2(fmaf(v[r + 2], p.c, -o4.z)) + fast_exp2(fmaf(v[r + 3], p.c, -o4.w)));
+    }
+  } else {            // window key: row r (window row r % w) sees it when key <= P + r % w
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const int row = r0 + r;
+      if (row < p.R && key <= P + row % p.w) acc8[r & 7] += fast_exp2(fmaf(v[r], p.c, -off[row]));
+    }
+  }
+}
+
 // --------------------------------------------------------------------------
 // shared body: producer + MMA roles are identical for both passes, only the
 // operand order of the MMA and the epilogue differ.
@@ -208,64 +260,34 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, TcParams p) {
       const int buf = t & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (t >> 1) & 1))) { *cta_err = 1; break; }
       tc_fence_after();
-      float v[128];
       const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + buf * 128;
-      tmem_ld32(taddr + 0, v);
-      tmem_ld32(taddr + 32, v + 32);
-      tmem_ld32(taddr + 64, v + 64);
-      tmem_ld32(taddr + 96, v + 96);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
       const int key0 = key_begin + t * kBN;
-      if (!kScorePass) {
-        // row my_lane: keys key0 .. key0+127
-        const bool full_vis = (key0 + kBN - 1 <= P) && (key0 + kBN <= key_end);
-        float tmax = kNegInf;
-        if (full_vis) {
+      // 32-column chunks, double-buffered: the load of chunk q+1 is in flight
+      // while chunk q is reduced
+      float va[32], vb[32];
+      float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      tmem_ld32(taddr, va);
+      tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 128; ++j) { v[j] *= p.c; tmax = fmaxf(tmax, v[j]); }
+      for (int q = 0; q < 4; ++q) {
+        float *cur = (q & 1) ? vb : va;
+        float *nxt = (q & 1) ? va : vb;
+        if (q < 3) tmem_ld32(taddr + 32 * (q + 1), nxt);
+        if (q == 3) {              // every column of this buffer has been read
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+        }
+        if (!kScorePass) {
+          epi_stats_chunk(cur, key0 + 32 * q, key_end, P, row_pos, p.c, m, l);
         } else {
-#pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            const int key = key0 + j;
-            v[j] = (key < key_end && key <= row_pos) ? v[j] * p.c : kNegInf;
-            tmax = fmaxf(tmax, v[j]);
-          }
+          epi_score_chunk(cur, off, 32 * q, key0 + my_lane, P, p, acc8);
         }
-        const float mn = fmaxf(m, tmax);
-        const float ms = (mn == kNegInf) ? 0.f : mn;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 128; j += 4) {
-          s0 += fast_exp2(v[j] - ms);
-          s1 += fast_exp2(v[j + 1] - ms);
-          s2 += fast_exp2(v[j + 2] - ms);
-          s3 += fast_exp2(v[j + 3] - ms);
-        }
-        l = l * fast_exp2(m - ms) + ((s0 + s1) + (s2 + s3));
-        m = mn;
-      } else {
-        // key key0 + my_lane: rows 0..127
+        if (q < 3) tmem_wait_ld();
+      }
+      if (kScorePass) {
         const int key = key0 + my_lane;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-        if (key <= P) {
-#pragma unroll
-          for (int r = 0; r < 128; r += 4) {
-            const float4 o4 = *reinterpret_cast<const float4 *>(off + r);
-            s0 += fast_exp2(fmaf(v[r], p.c, -o4.x));
-            s1 += fast_exp2(fmaf(v[r + 1], p.c, -o4.y));
-            s2 += fast_exp2(fmaf(v[r + 2], p.c, -o4.z));
-            s3 += fast_exp2(fmaf(v[r + 3], p.c, -o4.w));
-          }
-        } else {
-          // window key: row r (window row r % w) sees it when key <= P + r % w
-#pragma unroll
-          for (int r = 0; r < 128; ++r) {
-            if (r < p.R && key <= P + r % p.w) s0 += fast_exp2(fmaf(v[r], p.c, -off[r]));
-          }
-        }
-        if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = (s0 + s1) + (s2 + s3);
+        const float sum = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+        if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = sum;
       }
     }
     if (!kScorePass && my_lane < p.R)

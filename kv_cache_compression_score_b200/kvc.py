@@ -37,8 +37,8 @@ SIGNATURES = {
     "kvc_tsp_select_gather": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p, _c_int, _c_p,
                                        _c_p, _c_p, _c_sz, _c_p]),
     "kvc_gqa_decode_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
-    "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_p, _c_p,
-                                     _c_int, _c_p, _c_p, _c_sz, _c_p]),
+    "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_i64, _c_p,
+                                     _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
 }
 
 _lib = None
@@ -165,5 +165,6 @@ def kvc_gqa_decode_attn(q, k_c, v_c, kv_row_offset, kv_len, max_kv_len: int, sca
                         stream=None) -> None:
     batch, n_h, d_h = q.shape
     _check(lib().kvc_gqa_decode_attn(dtype_code(q), batch, n_h, k_c.shape[1], d_h, scale, _dptr(q), _dptr(k_c),
-                                     _dptr(v_c), _dptr(kv_row_offset), _dptr(kv_len), max_kv_len, _dptr(out),
+                                     _dptr(v_c), k_c.shape[0], _dptr(kv_row_offset), _dptr(kv_len), max_kv_len,
+                                     _dptr(out),
                                      _dptr(ws), ws.numel() * ws.element_size(), _stream(stream)))

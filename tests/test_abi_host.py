@@ -112,12 +112,14 @@ def test_select_gather_decode_tsp_reject_before_launch(L):
     assert L.kvc_gather_kv(kvc.KVC_BF16, 2, slp, P16, P16, 8, 4, 64, P16, P16, P16, P16, P16, None) == UNSUPPORTED
     assert L.kvc_gather_kv(kvc.KVC_BF16, 2, slp, P16, P16, 8, 128, 64, P16, P16, P8, P16, P16, None) == INVALID
     # decode: group of 3, odd head dim, small workspace
-    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 24, 8, 128, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 1 << 30,
-                                 None) == UNSUPPORTED
-    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 80, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 1 << 30,
-                                 None) == UNSUPPORTED
-    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 128, 0.0, P16, P16, P16, P16, P16, 100, P16, P16, 8,
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 24, 8, 128, 0.0, P16, P16, P16, 200, P16, P16, 100, P16, P16,
+                                 1 << 30, None) == UNSUPPORTED
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 80, 0.0, P16, P16, P16, 200, P16, P16, 100, P16, P16,
+                                 1 << 30, None) == UNSUPPORTED
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 128, 0.0, P16, P16, P16, 200, P16, P16, 100, P16, P16, 8,
                                  None) == WORKSPACE
+    assert L.kvc_gqa_decode_attn(kvc.KVC_BF16, 2, 32, 8, 128, 0.0, P16, P16, P16, 0, P16, P16, 100, P16, P16,
+                                 1 << 30, None) == INVALID
     # TSP: k_tsp beyond the prefix, even pool
     assert L.kvc_tsp_select_gather(kvc.KVC_BF16, 100, 8, 32, 7, 69, P16, P16, 4096, P16, P16, P16, 1 << 20,
                                    None) == INVALID

@@ -1,0 +1,92 @@
+"""Parity at the full workload sizes, in the launch configuration the bench
+uses.  The fp64 oracle computes every output of these sizes, so the whole
+output is compared (not a sample).
+
+Workloads (seeded synthetic stand-ins for the pages' long-context models):
+  Llama-3-8B-shaped layer: n_h 32, n_kv 8, d_h 128, bf16, S 32768, window 32,
+      pool 7, budget 2048, 1% of keys boosted; decode batch 16;
+  long context: S 131072, budget 4096 and budget S (identity);
+  FastKV TSP layer: S 32768, k_tsp = floor(0.2 S), hidden [S, 4096] bf16,
+      then the first propagated layer at S' = k_tsp + 32 with budget
+      floor(0.1 S);
+  ragged: 16 lengths uniform on [4096, 65536], budget 1024.
+"""
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_compression_score_b200 import synth
+from kv_cache_compression_score_b200.runner import TspSelector, from_device, to_device
+from oracle import kvc_oracle as O
+from parity_helpers import run_and_check_compress, run_and_check_decode
+
+pytestmark = pytest.mark.gpu
+
+N_H, N_KV, D, W, POOL = 32, 8, 128, 32, 7
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _built():
+    from kv_cache_compression_score_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def test_llama8b_layer_s32k():
+    r = run_and_check_compress("bf16", [32768], N_H, N_KV, D, W, POOL, 2048, seed=1002, boost_frac=0.01)
+    # decode at batch 16 over 16 compact caches of 2048 rows (the step's own cache first)
+    kc = [from_device(r["comp"].buf.k_c)]
+    vc = [from_device(r["comp"].buf.v_c)]
+    for b in range(1, 16):
+        k, v = synth.keys_values(1009, b, 2048, N_KV, D, "bf16")
+        kc.append(k)
+        vc.append(v)
+    q = synth.decode_queries(1010, 16, N_H, D, "bf16")
+    run_and_check_decode("bf16", q, np.concatenate(kc), np.concatenate(vc), np.arange(16) * 2048, [2048] * 16, N_KV)
+
+
+@pytest.mark.parametrize("budget", [4096, 131072])
+def test_long_context_s128k(budget):
+    S = 131072
+    r = run_and_check_compress("bf16", [S], N_H, N_KV, D, W, POOL, budget, seed=1003, boost_frac=0.01)
+    if budget >= S:
+        # identity: every position kept, compact cache == cache, decode == full attention
+        np.testing.assert_array_equal(r["idx_g"], np.broadcast_to(np.arange(S), (N_KV, S)))
+        assert np.array_equal(from_device(r["comp"].buf.k_c), r["bt"]["k"])
+        q = synth.decode_queries(1011, 8, N_H, D, "bf16")
+        run_and_check_decode("bf16", q, r["bt"]["k"], r["bt"]["v"], [0] * 8, [S] * 8, N_KV)
+    else:
+        q = synth.decode_queries(1012, 8, N_H, D, "bf16")
+        run_and_check_decode("bf16", q, from_device(r["comp"].buf.k_c), from_device(r["comp"].buf.v_c), [0] * 8,
+                             [budget] * 8, N_KV)
+
+
+def test_fastkv_tsp_layer_and_next_layer():
+    S = 32768
+    k_tsp, kv_budget = O.rate_count(0.2, S), O.rate_count(0.1, S)
+    r = run_and_check_compress("bf16", [S], N_H, N_KV, D, W, POOL, kv_budget, seed=1004 + 15, boost_frac=0.01)
+    hidden = synth.hidden_states(1004, S, 4096, "bf16")
+    sel = TspSelector(S, W, POOL, k_tsp, 4096, "bf16")
+    idx, hout = sel.run(r["comp"].buf.scores_raw, to_device(hidden, "bf16"))
+    torch.cuda.synchronize()
+    idx_o = O.tsp_select(r["raw_o"], S, W, POOL, k_tsp)
+    pooled_o = O.tsp_pooled(r["raw_o"], S, W, POOL)
+    g = idx.cpu().numpy()
+    assert len(g) == k_tsp + W and np.all(np.diff(g) > 0)
+    np.testing.assert_array_equal(g[k_tsp:], np.arange(S - W, S))
+    kth = np.sort(pooled_o)[::-1][k_tsp - 1]
+    diff = set(g[:k_tsp].tolist()) ^ set(idx_o[:k_tsp].tolist())
+    assert all(abs(pooled_o[j] - kth) <= 1e-5 * kth for j in diff)
+    same = np.where(g == idx_o)[0]
+    assert np.array_equal(from_device(hout)[same], hidden[idx_o[same]])
+    # first layer after the TSP layer runs on S' = k_tsp + w tokens, same KV budget
+    run_and_check_compress("bf16", [k_tsp + W], N_H, N_KV, D, W, POOL, kv_budget, seed=1004 + 16, boost_frac=0.01)
+
+
+def test_ragged_16_sequences():
+    lens = synth.ragged_lengths(1005, 16, 4096, 65536)
+    r = run_and_check_compress("bf16", lens, N_H, N_KV, D, W, POOL, 1024, seed=1005, boost_frac=0.01)
+    cb = O.budget_offsets(lens, 1024)
+    q = synth.decode_queries(1013, 16, N_H, D, "bf16")
+    run_and_check_decode("bf16", q, from_device(r["comp"].buf.k_c), from_device(r["comp"].buf.v_c), cb[:-1],
+                         np.diff(cb), N_KV)
