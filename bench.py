@@ -11,7 +11,8 @@ pool 7, budget 2048, 1% of keys boosted):
 
 value = K tokens/s of score + select + gather (S / time / 1e3), whole job over
 all ranks; decode GB/s and the per-call breakdown are extra keys.  Timing: CUDA
-events around every step on the launching stream, L2 flushed (256 MiB write)
+events around every step on the launching stream, L2 flushed (256 MiB write,
+then a 256 MiB read sweep so no dirty lines are left)
 between steps outside the events, max over ranks.  With N > 1 every rank runs
 its own sequences (weak scaling, no collective on the data path).
 
@@ -150,7 +151,17 @@ def run_ours(args):
     off = torch.arange(nb, dtype=torch.int64, device=dev) * B
     ln = torch.full((nb,), B, dtype=torch.int32, device=dev)
     dec = Decoder(nb, n_h, n_kv, d, B, device=dev)
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)    # 256 MiB > 2x L2
+    # L2 flush between steps: write 256 MiB (> 2x L2), then read another
+    # 256 MiB so the timed step starts from a cache holding none of its data and
+    # no dirty lines waiting to be written back
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sweep = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        torch.sum(sweep, dim=0, out=sink)
+
     stream = torch.cuda.current_stream(dev)
 
     def step(evs=None):
@@ -165,7 +176,7 @@ def run_ours(args):
         if evs: evs[4].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize()
     assert comp.device_error_word() == 0, "device error word set"
@@ -178,7 +189,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         step(evs[i])
     torch.cuda.synchronize()
     if world > 1:
@@ -197,7 +208,7 @@ def run_ours(args):
         t_ssg, t_step, t_dec = tt.tolist()
 
     # ---- e2e: the same path through the C ABI with pinned host buffers
-    e2e = run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush)
+    e2e = run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush_l2)
     if world > 1:
         tt = torch.tensor([e2e["t_ms"]], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -228,7 +239,7 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1), 1% keys boosted +3 sigma)",
             "config": {"workload": cfg["name"], "n_h": n_h, "n_kv": n_kv, "d_h": d, "seq_len": S, "window": w,
                        "pool": cfg["pool_k"], "budget": B, "decode_batch": nb,
-                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "l2": "flushed between steps (256 MiB write + 256 MiB read sweep, outside the timed events)",
                        "parallelism": f"replicas x{world}"},
             "gbs": round(ssg_gbs, 1),
             "decode": {"gbs": round(dec_gbs, 1), "us": round(t_dec * 1e3, 2), "frac_of_8000": round(dec_gbs / 8000, 3)},
@@ -251,7 +262,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush):
+def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush_l2):
     """Inputs copied host->device from pinned memory and results device->host
     inside the timed region, every step."""
     import torch
@@ -267,7 +278,7 @@ def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, 
     n = max(3, min(args.steps, 10))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n + 1)]
     for i in range(n + 1):             # first iteration untimed (warm-up)
-        flush.zero_()
+        flush_l2()
         evs[i][0].record(stream)
         d_q.copy_(h_q, non_blocking=True)
         d_k.copy_(h_k, non_blocking=True)

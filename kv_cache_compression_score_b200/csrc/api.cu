@@ -125,15 +125,11 @@ kvc_status plan_decode(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, int 
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVC_ERR_UNSUPPORTED, "GQA group %d not in {1,2,4,8}", G);
   if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
   if (max_kv_len < 0) return fail(KVC_ERR_INVALID_ARG, "max_kv_len must be >= 0");
-  // chunks of whole tiles such that the persistent grid (2 CTAs per SM) gets
-  // about six work items per CTA
+  // stream-K over warps: every (batch entry, KV head) unit gets at most
+  // decode_slots(max_kv_len) partial slots
   const int64_t units = (int64_t)batch * n_kv;
-  const int tile = kvc::decode_tile_rows();
-  const int64_t target_items = 6 * 2 * kvc::kNumSMs;
-  int64_t rows = (int64_t)max_kv_len * units / target_items;
-  rows = std::max<int64_t>(2 * tile, (rows + tile - 1) / tile * tile);
-  pl->chunk_rows = (int)rows;
-  pl->n_chunks = std::max(1, (int)((max_kv_len + rows - 1) / rows));
+  pl->chunk_rows = 0;
+  pl->n_chunks = kvc::decode_slots(max_kv_len);
   pl->off_tickets = kErrWordBytes;
   pl->off_part = round_up(pl->off_tickets + (size_t)units * sizeof(int), 256);
   pl->bytes = pl->off_part + (size_t)units * pl->n_chunks * G * (d_h + 2) * sizeof(float);

@@ -4,343 +4,398 @@
 // section 1; "Variantes de l'attention et compression du cache KV",
 // introduction).
 //
-// Persistent CTAs (2 per SM) walk the work items (batch entry, KV head, chunk
-// of rows) grid-stride.  Warp 4 is a TMA producer: for every 32-row tile of
-// an item it loads the head's K and V rows (NHD layout, 3-D tensor maps, no
-// swizzle, no multicast) into a ring of shared-memory stages.  Warps 0-3
-// consume: a row of d_h elements is split over LPR = d_h / 16 lanes (16
-// elements each, read as 16-byte chunks that are contiguous across a quarter
-// warp), the G query heads of h sit in registers pre-scaled to log2 units,
-// logits are reduced over the LPR lanes with xor-shuffles and every row group
-// keeps an online softmax.  At the end of an item row groups and warps are
-// merged; the item's partial (m, l, acc) goes to the workspace, and the last
-// item of a (b, h) to finish (atomic ticket, no waiting) merges all partials.
-#include <cuda.h>
-
+// Work split (stream-K over warps): the rows of all (batch entry, KV head)
+// units are laid end to end and every warp of the grid takes an equal
+// contiguous slice, so the load is balanced to a row whatever the lengths.
+// A slice covers one or a few unit segments; each segment yields a partial
+// (m, l, acc) and the last warp to finish a unit (atomic ticket, no waiting)
+// merges its partials into the output.
+//
+// Per warp: a row of d_h elements is split over LPR = d_h / 16 lanes (16
+// elements each), RPW = 32 / LPR rows per step.  Each lane prefetches the K
+// and V bytes it will read itself with 16-byte cp.async into a private ring
+// (so no cross-lane synchronisation is needed), computes its G query-head
+// partial dot products (fma.rn.f32x2), reduces them over the LPR lanes with
+// xor-shuffles and keeps an online softmax whose reference max is only moved,
+// by warp vote, when a logit exceeds it by more than kSlack (log2 units):
+// p = 2^(s - m) <= 2^kSlack never overflows and the rare rescale is
+// warp-uniform.
 #include "kvc_common.cuh"
 #include "kvc_internal.h"
 
 namespace kvc {
 namespace {
 
-constexpr int kConsumers = 4;                       // consumer warps
-constexpr int kThreadsDec = (kConsumers + 1) * 32;  // + one producer warp
-constexpr int kRS = 32;                             // rows per tile
+constexpr int kWarps = 8;                 // warps per CTA
+constexpr int kThreadsDec = kWarps * 32;
+constexpr float kSlack = 8.f;             // log2 headroom before the reference max moves
+constexpr int kMinRowsPerWarp = 32;
 
-template <typename T, int D>
-struct DecLayout {
-  static constexpr int kEsz = sizeof(T);
-  static constexpr int kTile = kRS * D * kEsz;                    // K or V tile bytes
-  static constexpr int kStages = (96 * 1024) / (2 * kTile) < 6 ? (96 * 1024) / (2 * kTile) : 6;
-  static constexpr int kOffBar = kStages * 2 * kTile;
-  static constexpr int kOffMl = kOffBar + 2 * 8 * 8;              // up to 8 stages x 2 barriers
-  static constexpr int kBytesTiles = kOffMl;
+template <typename T>
+struct DecRing {
+  static constexpr int kNch = (int)sizeof(T);                 // 16-byte chunks per lane and row (16 elements)
+  static constexpr int kLaneBytes = kNch * 16 * 2;             // K + V of one row slice
+  static constexpr int kStepBytes = 32 * kLaneBytes;           // whole warp
+  static constexpr int kDepth = (96 * 1024) / (kWarps * kStepBytes) * 2 > 12 ? 12
+                                : (96 * 1024) / (kWarps * kStepBytes) * 2;   // 12 (bf16) or 6 (fp32)
+  static constexpr int kSmem = kWarps * kDepth * kStepBytes;   // 192 KB
 };
 
 struct DecParams {
-  const void *q;
+  const void *q, *kc, *vc;
   const int64_t *row_off;
   const int *kv_len;
   float *out;
   float *part;
   int *tickets;
-  int *err;
-  int batch, n_h, n_kv, n_chunks, chunk_rows;
-  float c;   // scale * log2(e)
+  int batch, n_h, n_kv, slots;   // slots: partial slots per unit
+  float c;                       // scale * log2(e)
 };
 
-KVC_DEVINL void merge_scale(float m, float m2, float &s1, float &s2, float &mn) {
-  mn = fmaxf(m, m2);
-  if (mn == kNegInf) { s1 = 0.f; s2 = 0.f; return; }
-  s1 = fast_exp2(m - mn);
-  s2 = fast_exp2(m2 - mn);
+KVC_DEVINL void ffma2(float &a0, float &a1, float x0, float x1, float y0, float y1) {
+  uint64_t d;
+  const uint64_t a = ((uint64_t)__float_as_uint(a1) << 32) | __float_as_uint(a0);
+  const uint64_t x = ((uint64_t)__float_as_uint(x1) << 32) | __float_as_uint(x0);
+  const uint64_t y = ((uint64_t)__float_as_uint(y1) << 32) | __float_as_uint(y0);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(x), "l"(y), "l"(a));
+  a0 = __uint_as_float((uint32_t)d);
+  a1 = __uint_as_float((uint32_t)(d >> 32));
 }
 
 template <typename T> KVC_DEVINL void unpack16(const uint4 &v, float *o);
 template <> KVC_DEVINL void unpack16<__nv_bfloat16>(const uint4 &v, float *o) { Elem<__nv_bfloat16>::unpack(v, o); }
 template <> KVC_DEVINL void unpack16<float>(const uint4 &v, float *o) { Elem<float>::unpack(v, o); }
 
+KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+
+// warp w's slice of the flattened row space is [start(w), start(w + 1))
+KVC_DEVINL int64_t slice_start(int64_t w, int64_t R, int64_t NW) { return w * R / NW; }
+// the warp whose slice contains global row x (0 <= x < R)
+KVC_DEVINL int64_t owner(int64_t x, int64_t R, int64_t NW) {
+  int64_t w = x * NW / R;
+  while (w + 1 < NW && slice_start(w + 1, R, NW) <= x) ++w;
+  while (w > 0 && slice_start(w, R, NW) > x) --w;
+  return w;
+}
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreadsDec)
-gqa_decode_tma(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, DecParams p) {
-  using L = DecLayout<T, D>;
-  constexpr int LPR = D / 16;                 // lanes per row
-  constexpr int RPW = 32 / LPR;               // rows per warp step
-  constexpr int kSteps = kRS / (kConsumers * RPW);
-  constexpr int EPC = 16 / L::kEsz;           // elements per 16-byte chunk
-  constexpr int NCH = 16 / EPC;               // chunks per lane (16 elements)
-  static_assert(kSteps >= 1 && kRS % (kConsumers * RPW) == 0, "tile rows");
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-  uint64_t *empty = full + 8;
-  float *sm_ml = reinterpret_cast<float *>(smem + L::kOffMl);            // [warps][G][2]
-  float *sm_acc = sm_ml + kConsumers * G * 2;                            // [warps][G][D]
-  int *sm_flag = reinterpret_cast<int *>(sm_acc + kConsumers * G * D);   // [0] last, [1] error
-
+__global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p) {
+  using RG = DecRing<T>;
+  constexpr int LPR = D / 16;              // lanes per row
+  constexpr int RPW = 32 / LPR;            // rows per warp step
+  constexpr int EPC = 16 / (int)sizeof(T); // elements per 16-byte chunk
+  constexpr int NCH = RG::kNch;
+  constexpr int kRing = RG::kDepth;
+  static_assert(NCH * EPC == 16, "16 elements per lane");
+  extern __shared__ uint4 smem_v4[];
+  uint8_t *smem_raw = reinterpret_cast<uint8_t *>(smem_v4);
   const int warp = warp_id(), lane = lane_id();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < L::kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kConsumers); }
-    sm_flag[1] = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmk);
-    tma_prefetch_desc(&tmv);
-  }
-  __syncthreads();
+  // ring of kRing steps per warp; within a step, 16-byte chunk j of lane L sits
+  // at (j * 32 + L) * 16 so a quarter warp touches 128 consecutive bytes
+  uint8_t *ring = smem_raw + warp * kRing * RG::kStepBytes + lane * 16;
+  const int rg = lane / LPR, sl = lane % LPR;
+  const int n_units = p.batch * p.n_kv;
 
-  const int n_items = p.batch * p.n_kv * p.n_chunks;
-  if (warp == kConsumers) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int t = 0;
-      volatile int *vflag = sm_flag;
-      for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-        const int c = it % p.n_chunks, bh = it / p.n_chunks, h = bh % p.n_kv, b = bh / p.n_kv;
-        const int len = p.kv_len[b], r0 = c * p.chunk_rows;
-        if (r0 >= len) continue;
-        const int r1 = min(len, r0 + p.chunk_rows);
-        const int64_t o = p.row_off[b];
-        for (int row = r0; row < r1; row += kRS, ++t) {
-          const int s = t % L::kStages;
-          if (!vflag[1] && !mbar_wait(&empty[s], ((t / L::kStages) & 1) ^ 1)) vflag[1] = 1;
-          mbar_expect_tx(&full[s], 2 * L::kTile);
-          uint8_t *ks = smem + s * 2 * L::kTile;
-          tma_load_3d(ks, &tmk, &full[s], 0, h, (int)(o + row));
-          tma_load_3d(ks + L::kTile, &tmv, &full[s], 0, h, (int)(o + row));
-        }
-      }
-      for (int u = max(0, t - L::kStages); u < t; ++u)      // drain copies in flight
-        if (!mbar_wait(&full[u % L::kStages], (u / L::kStages) & 1)) { vflag[1] = 1; break; }
-    }
-  } else {
-    // ------------------------------------------------------------ consumers
-    const int rg = lane / LPR, sl = lane % LPR;
-    volatile int *vflag = sm_flag;
-    int t = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-      const int c = it % p.n_chunks, bh = it / p.n_chunks, h = bh % p.n_kv, b = bh / p.n_kv;
-      const int len = p.kv_len[b], r0 = c * p.chunk_rows;
-      const int n_active = (len + p.chunk_rows - 1) / p.chunk_rows;
-      float *outp = p.out + ((size_t)b * p.n_h + (size_t)h * G) * D;
-      if (len == 0) {
-        if (c == 0)
-          for (int e = threadIdx.x; e < G * D; e += kConsumers * 32) outp[e] = 0.f;
-        continue;
-      }
-      if (r0 >= len) continue;
-      const int r1 = min(len, r0 + p.chunk_rows);
+  // ---- the flattened row space and this warp's slice
+  int64_t R = 0;
+  for (int b = 0; b < p.batch; ++b) R += (int64_t)p.kv_len[b] * p.n_kv;
+  const int64_t NW_all = (int64_t)gridDim.x * kWarps;
+  const int64_t NW = R > 0 ? min(NW_all, max((int64_t)1, R / kMinRowsPerWarp)) : 0;
+  const int64_t gw = (int64_t)blockIdx.x * kWarps + warp;
 
-      // query slices: element d = j * (LPR * EPC) + sl * EPC + i of chunk j
-      float qr[G][16];
-      const T *qb = static_cast<const T *>(p.q) + ((size_t)b * p.n_h + (size_t)h * G) * D;
+  // units of empty caches produce zeros (first warp of the grid)
+  if (gw == 0)
+    for (int u = 0; u < n_units; ++u)
+      if (p.kv_len[u / p.n_kv] == 0)
+        for (int e = lane; e < G * D; e += 32)
+          p.out[((size_t)(u / p.n_kv) * p.n_h + (size_t)(u % p.n_kv) * G) * D + e] = 0.f;
+  if (gw >= NW) return;
+
+  int64_t x = slice_start(gw, R, NW);
+  const int64_t x_end = slice_start(gw + 1, R, NW);
+  // locate the unit containing row x
+  int b = 0;
+  int64_t base_b = 0;
+  while (base_b + (int64_t)p.kv_len[b] * p.n_kv <= x) { base_b += (int64_t)p.kv_len[b] * p.n_kv; ++b; }
+
+  while (x < x_end) {
+    const int len = p.kv_len[b];
+    const int h = (int)((x - base_b) / len);
+    const int64_t u0 = base_b + (int64_t)h * len;           // unit start in the row space
+    const int r0 = (int)(x - u0);
+    const int r1 = (int)(min(x_end, u0 + len) - u0);
+    const int u = b * p.n_kv + h;
+
+    // query slices of the G heads of h: element d = j * (LPR * EPC) + sl * EPC + i of chunk j
+    float qr[G][16];
+    const T *qb = static_cast<const T *>(p.q) + ((size_t)b * p.n_h + (size_t)h * G) * D;
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        unpack16<T>(ld_nc16(qb + (size_t)g * D + j * (LPR * EPC) + sl * EPC), &qr[g][j * EPC]);
+#pragma unroll
+        for (int i = 0; i < EPC; ++i) qr[g][j * EPC + i] *= p.c;
+      }
+    float acc[G][16], m[G], l[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = kNegInf;
+      l[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[g][e] = 0.f;
+    }
+
+    const int64_t o = p.row_off[b];
+    const T *kb = static_cast<const T *>(p.kc) + ((size_t)o * p.n_kv + h) * D + sl * EPC;
+    const T *vb = static_cast<const T *>(p.vc) + ((size_t)o * p.n_kv + h) * D + sl * EPC;
+    const size_t rstride = (size_t)p.n_kv * D;
+    const int n_steps = (r1 - r0 + RPW - 1) / RPW;
+    // lane-private ring slot of step s: K chunks then V chunks, 16 B each
+#pragma unroll 1
+    for (int s = 0; s < kRing - 1 + n_steps; ++s) {
+      if (s < n_steps + kRing - 1) {
+        // prefetch step s (zero-filled past the segment); a group per step
+        const int row = r0 + s * RPW + rg;
+        const bool valid = s < n_steps && row < r1;
+        const size_t ro = (size_t)(valid ? row : r0) * rstride;
+        uint8_t *dst = ring + (s % kRing) * RG::kStepBytes;
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
-          unpack16<T>(ld_nc16(qb + (size_t)g * D + j * (LPR * EPC) + sl * EPC), &qr[g][j * EPC]);
-#pragma unroll
-          for (int i = 0; i < EPC; ++i) qr[g][j * EPC + i] *= p.c;
+          cp_async16(dst + j * 512, kb + ro + j * (LPR * EPC), valid);
+          cp_async16(dst + (NCH + j) * 512, vb + ro + j * (LPR * EPC), valid);
         }
-      float acc[G][16], m[G], l[G];
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      const int st = s - (kRing - 1);           // step consumed in this iteration
+      if (st < 0) continue;
+      asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
+      const uint8_t *src = ring + (st % kRing) * RG::kStepBytes;
+      const bool valid = r0 + st * RPW + rg < r1;
+      float kf[16];
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) unpack16<T>(*reinterpret_cast<const uint4 *>(src + j * 512), &kf[j * EPC]);
+      float sc[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        m[g] = kNegInf;
-        l[g] = 0.f;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[g][e] = 0.f;
+        for (int e = 0; e < 16; e += 4) {
+          ffma2(a0, a1, qr[g][e], qr[g][e + 1], kf[e], kf[e + 1]);
+          ffma2(a2, a3, qr[g][e + 2], qr[g][e + 3], kf[e + 2], kf[e + 3]);
+        }
+        sc[g] = (a0 + a1) + (a2 + a3);
       }
-
-      for (int row = r0; row < r1; row += kRS, ++t) {
-        const int s = t % L::kStages;
-        // after a give-up anywhere in the CTA nobody waits again: the loops
-        // still run to their end (results flagged invalid), so every warp
-        // reaches the named barriers below
-        const bool got = vflag[1] ? true : mbar_wait(&full[s], (t / L::kStages) & 1);
-        if (!__all_sync(0xffffffffu, got) && lane == 0) vflag[1] = 1;
-        const uint8_t *ks = smem + s * 2 * L::kTile;
-        const uint8_t *vs = ks + L::kTile;
+      if constexpr (G <= LPR) {
+        // reduce-scatter over the LPR lanes of the row: afterwards this lane
+        // holds the full logit of one head, hs = sl / (LPR / G)
 #pragma unroll
-        for (int st = 0; st < kSteps; ++st) {
-          const int lr = st * (kConsumers * RPW) + warp * RPW + rg;
-          const bool valid = row + lr < r1;
-          float kf[16];
-          const uint8_t *krow = ks + lr * D * L::kEsz + sl * 16;
+        for (int k = G, o = LPR / 2; k > 1; k >>= 1, o >>= 1) {
+          const bool up = (sl & o) != 0;
 #pragma unroll
-          for (int j = 0; j < NCH; ++j) unpack16<T>(*reinterpret_cast<const uint4 *>(krow + j * LPR * 16), &kf[j * EPC]);
-          float sc[G];
+          for (int j = 0; j < k / 2; ++j) {
+            const float mine = up ? sc[k / 2 + j] : sc[j];
+            const float other = up ? sc[j] : sc[k / 2 + j];
+            sc[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+          }
+        }
+#pragma unroll
+        for (int o = (LPR / G) / 2; o >= 1; o >>= 1) sc[0] += __shfl_xor_sync(0xffffffffu, sc[0], o);
+        const float s_my = sc[0];
+        const int src0 = rg * LPR;                     // lane of head g: src0 + g * (LPR / G)
+        // move this lane's reference max only when its logit exceeds it by kSlack
+        const bool need = valid && s_my > m[0] + kSlack;
+        if (__any_sync(0xffffffffu, need)) {
+          const float mn = valid ? fmaxf(m[0], s_my) : m[0];
+          const float a = (mn == kNegInf) ? 1.f : fast_exp2(m[0] - mn);
+          l[0] *= a;
+          m[0] = mn;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            float a0 = 0.f, a1 = 0.f;
+            const float ag = __shfl_sync(0xffffffffu, a, src0 + g * (LPR / G));
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              a0 = fmaf(qr[g][e], kf[e], a0);
-              a1 = fmaf(qr[g][e + 1], kf[e + 1], a1);
-            }
-            sc[g] = a0 + a1;
-          }
-#pragma unroll
-          for (int off = 1; off < LPR; off <<= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
-          if (valid) {
-            float vf[16];
-            const uint8_t *vrow = vs + lr * D * L::kEsz + sl * 16;
-#pragma unroll
-            for (int j = 0; j < NCH; ++j)
-              unpack16<T>(*reinterpret_cast<const uint4 *>(vrow + j * LPR * 16), &vf[j * EPC]);
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              if (sc[g] > m[g]) {
-                const float a = fast_exp2(m[g] - sc[g]);
-                l[g] *= a;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[g][e] *= a;
-                m[g] = sc[g];
-              }
-              const float pr = fast_exp2(sc[g] - m[g]);
-              l[g] += pr;
-#pragma unroll
-              for (int e = 0; e < 16; ++e) acc[g][e] = fmaf(pr, vf[e], acc[g][e]);
-            }
+            for (int e = 0; e < 16; ++e) acc[g][e] *= ag;
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        const float pr = valid ? fast_exp2(s_my - m[0]) : 0.f;
+        l[0] += pr;
+        float pg[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) pg[g] = __shfl_sync(0xffffffffu, pr, src0 + g * (LPR / G));
+        if (valid) {
+          float vf[16];
+#pragma unroll
+          for (int j = 0; j < NCH; ++j)
+            unpack16<T>(*reinterpret_cast<const uint4 *>(src + (NCH + j) * 512), &vf[j * EPC]);
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) ffma2(acc[g][e], acc[g][e + 1], pg[g], pg[g], vf[e], vf[e + 1]);
+        }
+      } else {
+        // more heads than lanes per row: every lane reduces every head
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1)
+#pragma unroll
+          for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
+        bool need = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) need |= valid && sc[g] > m[g] + kSlack;
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float mn = valid ? fmaxf(m[g], sc[g]) : m[g];
+            const float a = (mn == kNegInf) ? 1.f : fast_exp2(m[g] - mn);
+            l[g] *= a;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[g][e] *= a;
+            m[g] = mn;
+          }
+        }
+        if (valid) {
+          float vf[16];
+#pragma unroll
+          for (int j = 0; j < NCH; ++j)
+            unpack16<T>(*reinterpret_cast<const uint4 *>(src + (NCH + j) * 512), &vf[j * EPC]);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pr = fast_exp2(sc[g] - m[g]);
+            l[g] += pr;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) ffma2(acc[g][e], acc[g][e + 1], pr, pr, vf[e], vf[e + 1]);
+          }
+        }
       }
-      // merge the row groups of the warp (lanes holding the same slice)
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+    if constexpr (G <= LPR) {
+      // every lane of the row group takes the (m, l) of each head from its owner lane
+      const float m_my = m[0], l_my = l[0];
 #pragma unroll
-      for (int off = LPR; off < 32; off <<= 1)
+      for (int g = 0; g < G; ++g) {
+        m[g] = __shfl_sync(0xffffffffu, m_my, rg * LPR + g * (LPR / G));
+        l[g] = __shfl_sync(0xffffffffu, l_my, rg * LPR + g * (LPR / G));
+      }
+    }
+    // merge the row groups of the warp (lanes holding the same slice)
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m[g], off);
-          const float l2 = __shfl_xor_sync(0xffffffffu, l[g], off);
-          float s1, s2, mn;
-          merge_scale(m[g], m2, s1, s2, mn);
-          l[g] = l[g] * s1 + l2 * s2;
-          m[g] = mn;
+    for (int off = LPR; off < 32; off <<= 1)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float a2 = __shfl_xor_sync(0xffffffffu, acc[g][e], off);
-            acc[g][e] = acc[g][e] * s1 + a2 * s2;
-          }
+      for (int g = 0; g < G; ++g) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m[g], off);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l[g], off);
+        const float mn = fmaxf(m[g], m2);
+        const float s1 = (mn == kNegInf) ? 0.f : fast_exp2(m[g] - mn);
+        const float s2 = (mn == kNegInf) ? 0.f : fast_exp2(m2 - mn);
+        l[g] = l[g] * s1 + l2 * s2;
+        m[g] = mn;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a2 = __shfl_xor_sync(0xffffffffu, acc[g][e], off);
+          acc[g][e] = acc[g][e] * s1 + a2 * s2;
         }
-      // merge the consumer warps through shared memory
-      if (rg == 0) {
+      }
+
+    float *outp = p.out + ((size_t)b * p.n_h + (size_t)h * G) * D;
+    const int64_t first = owner(u0, R, NW), last = owner(u0 + len - 1, R, NW);
+    if (first == last) {
+      // this warp owns the whole unit
+      if (rg == 0)
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          if (sl == 0) { sm_ml[(warp * G + g) * 2] = m[g]; sm_ml[(warp * G + g) * 2 + 1] = l[g]; }
+        for (int g = 0; g < G; ++g)
 #pragma unroll
           for (int j = 0; j < NCH; ++j)
 #pragma unroll
             for (int i = 0; i < EPC; ++i)
-              sm_acc[(warp * G + g) * D + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i];
+              outp[g * D + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i] / l[g];
+    } else {
+      float *pp = p.part + ((size_t)u * p.slots + (size_t)(gw - first)) * (size_t)(G * (D + 2));
+      if (rg == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (sl == 0) { pp[g * (D + 2)] = m[g]; pp[g * (D + 2) + 1] = l[g]; }
+#pragma unroll
+          for (int j = 0; j < NCH; ++j)
+#pragma unroll
+            for (int i = 0; i < EPC; ++i) pp[g * (D + 2) + 2 + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i];
         }
       }
-      asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
-      float *my_part = p.part + ((size_t)bh * p.n_chunks + c) * (size_t)(G * (D + 2));
-      for (int e = threadIdx.x; e < G * D; e += kConsumers * 32) {
-        const int g = e / D, d = e % D;
-        float M = kNegInf;
-#pragma unroll
-        for (int wv = 0; wv < kConsumers; ++wv) M = fmaxf(M, sm_ml[(wv * G + g) * 2]);
-        float Ls = 0.f, A = 0.f;
-#pragma unroll
-        for (int wv = 0; wv < kConsumers; ++wv) {
-          const float mw = sm_ml[(wv * G + g) * 2];
-          if (mw == kNegInf) continue;
-          const float sc = fast_exp2(mw - M);
-          Ls = fmaf(sm_ml[(wv * G + g) * 2 + 1], sc, Ls);
-          A = fmaf(sm_acc[(wv * G + g) * D + d], sc, A);
-        }
-        if (n_active == 1) {
-          outp[e] = A / Ls;
-        } else {
-          my_part[g * (D + 2) + 2 + d] = A;
-          if (d == 0) { my_part[g * (D + 2)] = M; my_part[g * (D + 2) + 1] = Ls; }
-        }
-      }
-      if (n_active > 1) {
+      __threadfence();
+      __syncwarp();
+      int last_in = 0;
+      if (lane == 0) last_in = (atomicAdd(&p.tickets[u], 1) == (int)(last - first));
+      last_in = __shfl_sync(0xffffffffu, last_in, 0);
+      if (last_in) {
         __threadfence();
-        asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
-        if (threadIdx.x == 0) sm_flag[0] = (atomicAdd(&p.tickets[bh], 1) == n_active - 1);
-        asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");
-        if (sm_flag[0]) {
-          __threadfence();
-          const float *pp = p.part + (size_t)bh * p.n_chunks * (size_t)(G * (D + 2));
-          for (int e = threadIdx.x; e < G * D; e += kConsumers * 32) {
-            const int g = e / D, d = e % D;
-            float M = kNegInf;
-            for (int cc = 0; cc < n_active; ++cc) M = fmaxf(M, __ldcg(pp + (size_t)cc * G * (D + 2) + g * (D + 2)));
-            float Ls = 0.f, A = 0.f;
-            for (int cc = 0; cc < n_active; ++cc) {
-              const float *q0 = pp + (size_t)cc * G * (D + 2) + g * (D + 2);
-              const float sc = fast_exp2(__ldcg(q0) - M);
-              Ls = fmaf(__ldcg(q0 + 1), sc, Ls);
-              A = fmaf(__ldcg(q0 + 2 + d), sc, A);
-            }
-            outp[e] = A / Ls;
+        const int n_seg = (int)(last - first + 1);
+        const float *pu = p.part + (size_t)u * p.slots * (size_t)(G * (D + 2));
+        constexpr int kSeg = G * (D + 2);
+        // per-head maxima and normalisers, segments spread over the lanes
+        float Mg[G], Lg[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float mx = kNegInf;
+          for (int j = lane; j < n_seg; j += 32) mx = fmaxf(mx, __ldcg(pu + (size_t)j * kSeg + g * (D + 2)));
+          Mg[g] = warp_max(mx);
+          float ls = 0.f;
+          for (int j = lane; j < n_seg; j += 32) {
+            const float mj = __ldcg(pu + (size_t)j * kSeg + g * (D + 2));
+            if (mj != kNegInf) ls += __ldcg(pu + (size_t)j * kSeg + g * (D + 2) + 1) * fast_exp2(mj - Mg[g]);
           }
-          if (threadIdx.x == 0) p.tickets[bh] = 0;   // leave the counter zeroed for the next call
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o2);
+          Lg[g] = ls;
         }
+        // accumulators: lane covers D / 32 consecutive elements of every head
+        constexpr int EPL = D / 32;
+        float A[G][EPL];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) A[g][i] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < n_seg; ++j) {
+          const float *q0 = pu + (size_t)j * kSeg;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float mj = __ldcg(q0 + g * (D + 2));
+            const float wgt = (mj == kNegInf) ? 0.f : fast_exp2(mj - Mg[g]);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) A[g][i] = fmaf(__ldcg(q0 + g * (D + 2) + 2 + lane * EPL + i), wgt, A[g][i]);
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) outp[g * D + lane * EPL + i] = A[g][i] / Lg[g];
+        if (lane == 0) p.tickets[u] = 0;   // leave the counter zeroed for the next call
       }
-      asm volatile("bar.sync 1, %0;" :: "n"(kConsumers * 32) : "memory");   // smem reuse by the next item
+    }
+    // next segment: the rest of this unit's rows belong to later warps, or
+    // the next unit starts here
+    x = u0 + r1;
+    if (r1 == len && h == p.n_kv - 1 && x < x_end) {
+      base_b += (int64_t)len * p.n_kv;
+      ++b;
+      while (p.kv_len[b] == 0) ++b;   // x < x_end <= R: a non-empty entry follows
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0 && sm_flag[1]) atomicCAS(p.err, 0, 2);
-}
-
-// ---------------------------------------------------------------- host side
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                     const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                     CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                     CUtensorMapFloatOOBfill);
-
-PFN_encodeTiled encode_fn() {
-  static PFN_encodeTiled fn = nullptr;
-  if (!fn) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
-  }
-  return fn;
-}
-
-// cache [rows, n_kv, D] -> boxes of D elements x 1 head x kRS rows (rows past
-// the cache read as zero)
-bool cache_map(CUtensorMap *m, const void *base, int64_t rows, int n_kv, int D, bool bf16) {
-  PFN_encodeTiled enc = encode_fn();
-  if (!enc) return false;
-  const int esz = bf16 ? 2 : 4;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_kv, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)n_kv * D * esz};
-  cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)kRS};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base),
-             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T, int D, int G>
 cudaError_t launch(const DecodeArgs &a, cudaStream_t st) {
-  using L = DecLayout<T, D>;
-  CUtensorMap mk, mv;
-  const bool bf = a.dt == KVC_BF16;
-  if (!cache_map(&mk, a.k_c, a.cache_rows, a.n_kv, D, bf) || !cache_map(&mv, a.v_c, a.cache_rows, a.n_kv, D, bf))
-    return cudaErrorInvalidValue;
-  DecParams p;
-  p.q = a.q; p.row_off = a.row_off; p.kv_len = a.kv_len; p.out = a.out; p.part = a.part; p.tickets = a.tickets;
-  p.err = a.err; p.batch = a.batch; p.n_h = a.n_h; p.n_kv = a.n_kv; p.n_chunks = a.n_chunks;
-  p.chunk_rows = a.chunk_rows; p.c = a.scale * kLog2e;
-  const int smem = 1024 + L::kBytesTiles + (kConsumers * G * 2 + kConsumers * G * D + 4) * (int)sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(gqa_decode_tma<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = DecRing<T>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(gqa_decode_streamk<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int items = a.batch * a.n_kv * a.n_chunks;
-  const int grid = items < 2 * kNumSMs ? items : 2 * kNumSMs;
-  gqa_decode_tma<T, D, G><<<grid, kThreadsDec, smem, st>>>(mk, mv, p);
+  DecParams p;
+  p.q = a.q; p.kc = a.k_c; p.vc = a.v_c; p.row_off = a.row_off; p.kv_len = a.kv_len; p.out = a.out;
+  p.part = a.part; p.tickets = a.tickets; p.batch = a.batch; p.n_h = a.n_h; p.n_kv = a.n_kv;
+  p.slots = a.n_chunks; p.c = a.scale * kLog2e;
+  gqa_decode_streamk<T, D, G><<<kNumSMs, kThreadsDec, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -356,7 +411,10 @@ cudaError_t by_group(const DecodeArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int decode_tile_rows() { return kRS; }
+// Partial slots a unit can need: every warp slice holds at least
+// kMinRowsPerWarp rows, so a unit of len rows meets at most
+// len / kMinRowsPerWarp + 2 slices.
+int decode_slots(int max_kv_len) { return max_kv_len / kMinRowsPerWarp + 2; }
 
 cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st) {
   if (a.dt == KVC_F32) return a.d_h == 64 ? by_group<float, 64>(a, st) : by_group<float, 128>(a, st);

@@ -60,10 +60,11 @@ struct DecodeArgs {
   float *part;
   int *tickets;
   int *err;              // device error word
-  int64_t cache_rows;    // rows of k_c / v_c (tensor-map extent)
-  int n_chunks, chunk_rows;
+  int64_t cache_rows;    // rows of k_c / v_c
+  int n_chunks;          // partial slots per (batch entry, KV head)
+  int chunk_rows;        // unused by the stream-K kernel (kept 0)
 };
 cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
-int decode_tile_rows();
+int decode_slots(int max_kv_len);
 
 }  // namespace kvc

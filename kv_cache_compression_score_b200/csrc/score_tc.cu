@@ -10,52 +10,64 @@
 //   stats pass:  D[row][key] = Q_win[row] . K[key]   (M = 128 rows, N = 128 keys)
 //                one epilogue thread per TMEM lane = window row keeps the
 //                running max / sum of 2^(y - m) in registers;
-//   score pass:  D[key][row] = K[key] . Q_win[row]   (M = 128 keys, N = rows)
+//   score pass:  D[key][row] = K[key] . Q_win[row]   (M = 128 keys, N = 128 rows)
 //                one epilogue thread per TMEM lane = key sums 2^(y - off_r)
 //                over the rows, off_r = m_r + log2(l_r) merged from the
 //                stats partials.
 //
-// Warp roles (192 threads): warp 0 streams K tiles with TMA into a 4-stage
-// shared-memory ring (128-byte swizzle, no multicast), warp 1 owns tensor
-// memory and issues the MMAs (one thread), warps 2-5 are the epilogue.  The
-// accumulator is double-buffered in tensor memory (2 x 128 columns) so the
-// MMA of tile t+1 overlaps the epilogue of tile t.  Every wait is bounded;
-// a wait that gives up sets the device error word and the CTA drains.
-#include <cuda.h>
-
+// Warp roles (416 threads, one CTA per SM):
+//   warps 0-3   load K tiles (128 keys x d_h) with 16-byte cp.async straight
+//               into the 128-byte-swizzled K-major layout the MMA reads, a
+//               5-stage ring; 16-byte cp.async streams these strided head rows
+//               faster than tensor-map copies with 128-byte boxes.  Rows past
+//               the sequence are zero-filled (no read);
+//   warp 4      owns tensor memory (512 columns: four 128-column accumulators)
+//               and issues the MMAs from one thread;
+//   warps 5-12  epilogue: two warps per TMEM lane quarter, each reading half
+//               of the accumulator columns.
+// Every wait is bounded; a wait that gives up sets the device error word and
+// the CTA stops waiting (results are then flagged invalid, never a hang).
 #include "kvc_common.cuh"
 #include "kvc_internal.h"
 
 namespace kvc {
 namespace {
 
-constexpr int kBN = 128;        // keys per tile (MMA N in the stats pass, M in the score pass)
-constexpr int kRows = 128;      // window-block rows (padded)
-constexpr int kStages = 4;
-constexpr int kThreadsTC = 192;
-constexpr int kEpiWarp0 = 2;
+constexpr int kBN = 128;          // keys per tile
+constexpr int kRows = 128;        // window-block rows (padded)
+constexpr int kStages = 5;        // K ring depth
+constexpr int kLag = kStages - 1; // tiles in flight per loader thread
+constexpr int kAccBufs = 4;       // TMEM accumulators
+constexpr int kLoadWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kEpiWarp0 = 5;
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsTC = (kLoadWarps + 1 + kEpiWarps) * 32;
+constexpr int kXch = 8;           // half-column exchange slots (score pass)
 
 template <int D>
 struct TcLayout {
-  static constexpr int kAtoms = D / 64;                     // 128-byte swizzle atoms along d
   static constexpr int kQBytes = kRows * D * 2;              // window block
   static constexpr int kKBytes = kBN * D * 2;                // one K tile
   static constexpr int kAtomBytes = 128 * 128;               // 128 rows x 128 B
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffBar = kOffK + kStages * kKBytes;
-  static constexpr int kBarCount = 2 * kStages + 2 + 2 + 1;
-  static constexpr int kOffMisc = kOffBar + 128;           // 13 barriers need 104 bytes
-  static constexpr int kOffOff = kOffMisc + 16;             // score pass: off_r[128], 16-byte aligned
-  static constexpr int kBytes = kOffOff + kRows * 4;
-  static constexpr int kAlloc = kBytes + 1024;              // room to align the base to 1 KB
-  static_assert(kBarCount * 8 <= 128, "barrier area");
+  static constexpr int kBarCount = 2 * kStages + 2 * kAccBufs + 1 + kXch;
+  static constexpr int kOffMisc = kOffBar + 256;
+  static constexpr int kOffOff = kOffMisc + 16;              // off_r[128] (score pass)
+  static constexpr int kOffXch = kOffOff + kRows * 4;        // [kXch][128] (score) / m,l halves (stats)
+  static constexpr int kBytes = kOffXch + kXch * kBN * 4;
+  static constexpr int kAlloc = kBytes + 1024;               // room to align the base to 1 KB
+  static_assert(kBarCount * 8 <= 256, "barrier area");
   static_assert(kOffOff % 16 == 0, "off[] is read as float4");
   static_assert(kOffK % 1024 == 0 && kKBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
 
 struct TcParams {
   const __nv_bfloat16 *q_win;
+  const __nv_bfloat16 *k;
   const int *cu_seqlens;
   float2 *part;
   float *raw;
@@ -64,29 +76,32 @@ struct TcParams {
   float c;   // scale * log2(e)
 };
 
-// Q_win rows r = g * w + i of (b, h) into the 128-byte-swizzled K-major tile;
-// rows >= R are zero.  Generic-proxy writes, made visible to the tensor core
-// by fence.proxy.async before the MMA thread is released.
+// 16-byte cp.async, zero-filled (no global read) when !valid
+KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+
+// Q_win rows r = g * w + i of (b, h) into the 128-byte-swizzled K-major tile
+// with cp.async (all chunks in flight at once); rows >= R are zero-filled.
+// Completion, publication to the tensor core and the q_full arrive are done
+// by the caller together with its first K tiles.
 template <int D>
-KVC_DEVINL void stage_q(uint8_t *sq, const TcParams &p, int b, int h, int tid, int nthreads) {
+KVC_DEVINL void stage_q_async(uint8_t *sq, const TcParams &p, int b, int h, int tid, int nthreads) {
   constexpr int kChunks = D / 8;   // 16-byte chunks per row
+#pragma unroll 4
   for (int e = tid; e < kRows * kChunks; e += nthreads) {
     const int r = e / kChunks, ch = e % kChunks;
     const int atom = ch >> 3, c16 = ch & 7;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < p.R) {
-      const int g = r / p.w, i = r % p.w;
-      v = *reinterpret_cast<const uint4 *>(p.q_win + ((size_t)(b * p.w + i) * p.n_h + (size_t)h * p.G + g) * D + ch * 8);
-    }
-    *reinterpret_cast<uint4 *>(sq + atom * TcLayout<D>::kAtomBytes + r * 128 + ((c16 ^ (r & 7)) << 4)) = v;
+    const bool valid = r < p.R;
+    const int g = valid ? r / p.w : 0, i = valid ? r % p.w : 0;
+    const __nv_bfloat16 *src = p.q_win + ((size_t)(b * p.w + i) * p.n_h + (size_t)h * p.G + g) * D + ch * 8;
+    cp_async16(sq + atom * TcLayout<D>::kAtomBytes + r * 128 + ((c16 ^ (r & 7)) << 4), src, valid);
   }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-KVC_DEVINL void set_err(int *err, int code) { atomicCAS(err, 0, code); }
-
 // Stats-pass reduction of 32 logits of one window row (keys k0..k0+31):
-// online max / sum of 2^(c*z - m), masked keys (beyond the chunk end or the
+// online max / sum of 2^(c*z - m); masked keys (beyond the chunk end or the
 // row's causal limit) contribute nothing.
 KVC_DEVINL void epi_stats_chunk(float *v, int k0, int key_end, int P, int row_pos, float c, float &m, float &l) {
   if (!(k0 + 31 <= P && k0 + 32 <= key_end)) {
@@ -117,15 +132,14 @@ KVC_DEVINL void epi_stats_chunk(float *v, int k0, int key_end, int P, int row_po
 }
 
 // Score-pass accumulation for one key over window rows r0..r0+31:
-// acc += 2^(c*z_r - off_r), rows above the key's causal limit skipped.
-template <typename Params>
-KVC_DEVINL void epi_score_chunk(const float *v, const float *off, int r0, int key, int P, const Params &p,
+// acc += 2^(c*z_r - off_r); rows above the key's causal limit are skipped.
+KVC_DEVINL void epi_score_chunk(const float *v, const float *off, int r0, int key, int P, const TcParams &p,
                                 float *acc8) {
   if (key <= P) {     // prefix key (or the first window key): visible to every row
 #pragma unroll
     for (int r = 0; r < 32; r += 4) {
       const float4 o4 = *reinterpret_cast<const float4 *>(off + r0 + r);
-      acc8[(r >> 2) & 7] += fast_exp2(fmaf(v[r], p.c, -o4.x)) + fast_exp2(fmaf(v[r + 1], p.c, -o4.y)) +
+      acc8[(r >> 2) & 7] += (fast_exp2(fmaf(v[r], p.c, -o4.x)) + fast_exp2(fmaf(v[r + 1], p.c, -o4.y))) +
                             (fast_exp2(fmaf(v[r + 2], p.c, -o4.z)) + fast_exp2(fmaf(v[r + 3], p.c, -o4.w)));
     }
   } else {            // window key: row r (window row r % w) sees it when key <= P + r % w
@@ -137,13 +151,9 @@ KVC_DEVINL void epi_score_chunk(const float *v, const float *off, int r0, int ke
   }
 }
 
-// --------------------------------------------------------------------------
-// shared body: producer + MMA roles are identical for both passes, only the
-// operand order of the MMA and the epilogue differ.
-// --------------------------------------------------------------------------
 template <int D, bool kScorePass>
 __global__ void __launch_bounds__(kThreadsTC, 1)
-score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, TcParams p) {
+score_tc_kernel(TcParams p) {
   using L = TcLayout<D>;
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t0 = p.cu_seqlens[b], len = p.cu_seqlens[b + 1] - t0;
@@ -159,55 +169,73 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, TcParams p) {
   uint8_t *sk = smem + L::kOffK;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
   uint64_t *full = bars, *empty = bars + kStages;
-  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + 2, *q_full = acc_empty + 2;
+  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + kAccBufs;
+  uint64_t *q_full = acc_empty + kAccBufs;
+  uint64_t *xch_full = q_full + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
-  int *cta_err = reinterpret_cast<int *>(smem + L::kOffMisc + 4);
+  volatile int *cta_err = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
   float *off = reinterpret_cast<float *>(smem + L::kOffOff);
+  float *xch = reinterpret_cast<float *>(smem + L::kOffXch);
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], 4 * 32); }
-    mbar_init(q_full, 4 * 32);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], kLoadWarps * 32); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kAccBufs; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
+    mbar_init(q_full, kLoadWarps * 32);
+    for (int s = 0; s < kXch; ++s) mbar_init(&xch_full[s], 4);
     *cta_err = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmap_k);
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  if (warp == kMmaWarp) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int t = 0; t < n_tiles; ++t) {
+  if (warp < kLoadWarps) {
+    // ------------------------------------------------------------ K loaders
+    const int lt = threadIdx.x;                      // 0..127
+    stage_q_async<D>(sq, p, b, h, lt, kLoadWarps * 32);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    bool q_published = false;
+    constexpr int kChunks = kBN * D / 8;             // 16-byte chunks per tile
+    const uint8_t *kbase = reinterpret_cast<const uint8_t *>(p.k);
+    for (int t = 0; t < n_tiles + kLag; ++t) {
+      if (t < n_tiles) {
         const int s = t % kStages;
-        if (!mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1)) { *cta_err = 1; break; }
-        mbar_expect_tx(&full[s], L::kKBytes);
+        if (!*cta_err && !mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1)) *cta_err = 1;
         const int key0 = key_begin + t * kBN;
-#pragma unroll
-        for (int a = 0; a < L::kAtoms; ++a)
-          tma_load_3d(sk + s * L::kKBytes + a * L::kAtomBytes, &tmap_k, &full[s], a * 64, h, t0 + key0);
-        issued = t + 1;
+        uint8_t *dst = sk + s * L::kKBytes;
+#pragma unroll 4
+        for (int e = lt; e < kChunks; e += kLoadWarps * 32) {
+          const int row = e / (D / 8), ch = e % (D / 8);
+          const int atom = ch >> 3, c16 = ch & 7;
+          const bool valid = key0 + row < key_end;
+          const uint8_t *src = kbase + ((size_t)(t0 + (valid ? key0 + row : 0)) * p.n_kv + h) * (D * 2) + ch * 16;
+          cp_async16(dst + atom * L::kAtomBytes + row * 128 + ((c16 ^ (row & 7)) << 4), src, valid);
+        }
       }
-      // drain: every issued copy has landed before shared memory is released
-      for (int t = max(0, issued - kStages); t < issued; ++t)
-        if (!mbar_wait(&full[t % kStages], (t / kStages) & 1)) { *cta_err = 1; break; }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if (t >= kLag) {
+        // the window block (group 0) and tile t - kLag have landed for this
+        // thread: publish them to the tensor core
+        asm volatile("cp.async.wait_group %0;" :: "n"(kLag) : "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!q_published) { mbar_arrive(q_full); q_published = true; }
+        mbar_arrive(&full[(t - kLag) % kStages]);
+      }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-      bool ok = mbar_wait(q_full, 0);
-      int issued = 0;
       const uint32_t q_addr = smem_u32(sq), k_addr = smem_u32(sk);
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        const int s = t % kStages, buf = t & 1;
-        if (!mbar_wait(&full[s], (t / kStages) & 1)) { ok = false; break; }
-        if (!mbar_wait(&acc_empty[buf], ((t >> 1) & 1) ^ 1)) { ok = false; break; }
+      if (!mbar_wait(q_full, 0)) *cta_err = 1;
+      int issued = 0;
+      for (int t = 0; t < n_tiles && !*cta_err; ++t) {
+        const int s = t % kStages, buf = t % kAccBufs;
+        if (!mbar_wait(&full[s], (t / kStages) & 1)) { *cta_err = 1; break; }
+        if (!mbar_wait(&acc_empty[buf], ((t / kAccBufs) & 1) ^ 1)) { *cta_err = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 128;
 #pragma unroll
@@ -222,20 +250,21 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, TcParams p) {
         umma_commit(&acc_full[buf]);
         issued = t + 1;
       }
-      if (!ok) *cta_err = 1;
       // drain: the last commit tracks every MMA issued by this thread
-      if (issued > 0 && !mbar_wait(&acc_full[(issued - 1) & 1], ((issued - 1) >> 1) & 1)) *cta_err = 1;
+      if (issued > 0 && !mbar_wait(&acc_full[(issued - 1) % kAccBufs], ((issued - 1) / kAccBufs) & 1)) *cta_err = 1;
     }
   } else {
-    // ---------------------------------------------------------- epilogue
-    const int et = threadIdx.x - kEpiWarp0 * 32;        // 0..127
-    const int lane_base = 32 * (warp & 3);               // TMEM lanes this warp may access
-    const int my_lane = lane_base + lane;                // row (stats) or key (score)
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - kEpiWarp0;                 // 0..7
+    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..255
+    const int quarter = warp & 3;                    // TMEM lanes this warp may access
+    const int half = ew >> 2;                        // which 64 accumulator columns
+    const int my_lane = 32 * quarter + lane;         // row (stats) or key (score)
     if (kScorePass) {
       // merge the stats partials of every row into off_r = M + log2(L)
       const float2 *pp = p.part + (size_t)(b * p.n_kv + h) * p.n_chunks * kRows;
       const int nc = (len + p.keys_per_chunk - 1) / p.keys_per_chunk;
-      for (int r = et; r < kRows; r += 128) {
+      for (int r = et; r < kRows; r += kEpiWarps * 32) {
         float o = kPosInf;
         if (r < p.R) {
           float M = kNegInf;
@@ -249,95 +278,72 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, TcParams p) {
         }
         off[r] = o;
       }
+      asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
     }
-    stage_q<D>(sq, p, b, h, et, 128);
-    mbar_arrive(q_full);
-    if (kScorePass) asm volatile("bar.sync 1, 128;" ::: "memory");   // off[] visible to all epilogue warps
 
     float m = kNegInf, l = 0.f;
-    const int row_pos = P + (my_lane % max(p.w, 1));     // stats pass: this thread's row position
+    const int row_pos = P + (my_lane % max(p.w, 1));   // stats pass: this thread's row position
     for (int t = 0; t < n_tiles; ++t) {
-      const int buf = t & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (t >> 1) & 1))) { *cta_err = 1; break; }
+      const int buf = t % kAccBufs;
+      const bool got = *cta_err ? true : mbar_wait(&acc_full[buf], (t / kAccBufs) & 1);
+      if (!__all_sync(0xffffffffu, got) && lane == 0) *cta_err = 1;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)lane_base << 16) + buf * 128;
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * 128 + half * 64;
       const int key0 = key_begin + t * kBN;
-      // 32-column chunks, double-buffered: the load of chunk q+1 is in flight
-      // while chunk q is reduced
       float va[32], vb[32];
       float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       tmem_ld32(taddr, va);
       tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float *cur = (q & 1) ? vb : va;
-        float *nxt = (q & 1) ? va : vb;
-        if (q < 3) tmem_ld32(taddr + 32 * (q + 1), nxt);
-        if (q == 3) {              // every column of this buffer has been read
-          tc_fence_before();
-          mbar_arrive(&acc_empty[buf]);
-        }
-        if (!kScorePass) {
-          epi_stats_chunk(cur, key0 + 32 * q, key_end, P, row_pos, p.c, m, l);
-        } else {
-          epi_score_chunk(cur, off, 32 * q, key0 + my_lane, P, p, acc8);
-        }
-        if (q < 3) tmem_wait_ld();
-      }
+      tmem_ld32(taddr + 32, vb);
+      if (!kScorePass) epi_stats_chunk(va, key0 + half * 64, key_end, P, row_pos, p.c, m, l);
+      else epi_score_chunk(va, off, half * 64, key0 + my_lane, P, p, acc8);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);    // this warp's columns are read
+      if (!kScorePass) epi_stats_chunk(vb, key0 + half * 64 + 32, key_end, P, row_pos, p.c, m, l);
+      else epi_score_chunk(vb, off, half * 64 + 32, key0 + my_lane, P, p, acc8);
       if (kScorePass) {
-        const int key = key0 + my_lane;
         const float sum = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-        if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = sum;
+        const int slot = t % kXch;
+        const int key = key0 + my_lane;
+        if (half == 1) {
+          xch[slot * kBN + my_lane] = sum;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xch_full[slot]);
+        } else {
+          const bool ok = *cta_err ? true : mbar_wait(&xch_full[slot], (t / kXch) & 1);
+          if (!__all_sync(0xffffffffu, ok) && lane == 0) *cta_err = 1;
+          if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = sum + xch[slot * kBN + my_lane];
+        }
       }
     }
-    if (!kScorePass && my_lane < p.R)
-      p.part[((size_t)(b * p.n_kv + h) * p.n_chunks + c) * kRows + my_lane] = make_float2(m, l);
+    if (!kScorePass) {
+      // merge the two column halves of every row, then publish the partial
+      float *xm = xch, *xl = xch + kRows;
+      if (half == 1) { xm[my_lane] = m; xl[my_lane] = l; }
+      asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
+      if (half == 0 && my_lane < p.R) {
+        const float m2 = xm[my_lane], l2 = xl[my_lane];
+        const float mn = fmaxf(m, m2);
+        float ls = 0.f;
+        if (mn != kNegInf) ls = l * fast_exp2(m - mn) + l2 * fast_exp2(m2 - mn);
+        p.part[((size_t)(b * p.n_kv + h) * p.n_chunks + c) * kRows + my_lane] = make_float2(mn, ls);
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) { tc_fence_after(); tmem_dealloc(tmem_base, 256); }
-  if (threadIdx.x == 0 && *cta_err) set_err(p.err, 1);
-}
-
-// ---------------------------------------------------------- tensor maps
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                     const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                     CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                     CUtensorMapFloatOOBfill);
-
-PFN_encodeTiled get_encode() {
-  static PFN_encodeTiled fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_encodeTiled>(p);
-  }
-  return fn;
-}
-
-// K [T, n_kv, D] bf16 -> boxes of 64 d-elements x 1 head x 128 keys, 128-byte swizzle
-bool make_k_map(CUtensorMap *map, const void *k, int T, int n_kv, int D) {
-  PFN_encodeTiled enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_kv, (cuuint64_t)T};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)n_kv * D * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kBN};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (warp == kMmaWarp) { tc_fence_after(); tmem_dealloc(tmem_base, 512); }
+  if (threadIdx.x == 0 && *cta_err) atomicCAS(p.err, 0, 1);
 }
 
 template <int D>
 cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
-  CUtensorMap map;
-  if (!make_k_map(&map, a.k, a.T_total, a.n_kv, D)) return cudaErrorInvalidValue;
   TcParams p;
   p.q_win = static_cast<const __nv_bfloat16 *>(a.q_win);
+  p.k = static_cast<const __nv_bfloat16 *>(a.k);
   p.cu_seqlens = a.cu_seqlens;
   p.part = a.part;
   p.raw = a.raw;
@@ -352,9 +358,9 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(score_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
     return e;
   dim3 grid(a.n_chunks, a.n_kv, a.n_seqs);
-  score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(map, p);
+  score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(p);
   if ((e = cudaGetLastError())) return e;
-  score_tc_kernel<D, true><<<grid, kThreadsTC, smem, st>>>(map, p);
+  score_tc_kernel<D, true><<<grid, kThreadsTC, smem, st>>>(p);
   return cudaGetLastError();
 }
 
