@@ -6,6 +6,8 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
+#include <utility>
 #include <vector>
 
 #include "kvc_internal.h"
@@ -132,11 +134,27 @@ kvc_status plan_decode(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, int 
   pl->n_chunks = kvc::decode_slots(max_kv_len);
   pl->off_tickets = kErrWordBytes;
   pl->off_part = round_up(pl->off_tickets + (size_t)units * sizeof(int), 256);
-  pl->bytes = pl->off_part + (size_t)units * pl->n_chunks * G * (d_h + 2) * sizeof(float);
+  pl->bytes = pl->off_part + (size_t)units * pl->n_chunks * G * (d_h + 4) * sizeof(float);
   return KVC_OK;
 }
 
 }  // namespace
+
+namespace kvc {
+cudaError_t ensure_smem_limit(const void *fn, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<std::pair<const void *, int>, int>> done;   // ((fn, device), bytes)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto &d : done)
+    if (d.first.first == fn && d.first.second == dev && d.second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.push_back({{fn, dev}, bytes});
+  return e;
+}
+}  // namespace kvc
 
 extern "C" {
 

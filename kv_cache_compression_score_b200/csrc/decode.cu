@@ -36,10 +36,12 @@ struct DecRing {
   static constexpr int kNch = (int)sizeof(T);                 // 16-byte chunks per lane and row (16 elements)
   static constexpr int kLaneBytes = kNch * 16 * 2;             // K + V of one row slice
   static constexpr int kStepBytes = 32 * kLaneBytes;           // whole warp
-  static constexpr int kDepth = (96 * 1024) / (kWarps * kStepBytes) * 2 > 12 ? 12
-                                : (96 * 1024) / (kWarps * kStepBytes) * 2;   // 12 (bf16) or 6 (fp32)
-  static constexpr int kSmem = kWarps * kDepth * kStepBytes;   // 192 KB
+  static constexpr int kDepth = sizeof(T) == 2 ? 8 : 4;       // steps per warp (power of two)
+  static constexpr int kSmem = kWarps * kDepth * kStepBytes;   // 128 KB
 };
+
+// partial record of one segment and head: m, l, 2 pad words, acc[D]
+template <int D> constexpr int rec_floats() { return D + 4; }
 
 struct DecParams {
   const void *q, *kc, *vc;
@@ -52,14 +54,12 @@ struct DecParams {
   float c;                       // scale * log2(e)
 };
 
+// (a0, a1) += (x0, x1) * (y0, y1) as one packed fp32x2 FMA
 KVC_DEVINL void ffma2(float &a0, float &a1, float x0, float x1, float y0, float y1) {
-  uint64_t d;
-  const uint64_t a = ((uint64_t)__float_as_uint(a1) << 32) | __float_as_uint(a0);
-  const uint64_t x = ((uint64_t)__float_as_uint(x1) << 32) | __float_as_uint(x0);
-  const uint64_t y = ((uint64_t)__float_as_uint(y1) << 32) | __float_as_uint(y0);
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(x), "l"(y), "l"(a));
-  a0 = __uint_as_float((uint32_t)d);
-  a1 = __uint_as_float((uint32_t)(d >> 32));
+  asm("{\n\t.reg .b64 x, y, a;\n\t"
+      "mov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\tmov.b64 a, {%0, %1};\n\t"
+      "fma.rn.f32x2 a, x, y, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
 }
 
 template <typename T> KVC_DEVINL void unpack16(const uint4 &v, float *o);
@@ -154,26 +154,31 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
     const T *vb = static_cast<const T *>(p.vc) + ((size_t)o * p.n_kv + h) * D + sl * EPC;
     const size_t rstride = (size_t)p.n_kv * D;
     const int n_steps = (r1 - r0 + RPW - 1) / RPW;
-    // lane-private ring slot of step s: K chunks then V chunks, 16 B each
+    const size_t step_stride = (size_t)RPW * rstride;
+    const T *k_any = kb + (size_t)r0 * rstride, *v_any = vb + (size_t)r0 * rstride;   // a valid dummy source
+    const T *kq = kb + (size_t)(r0 + rg) * rstride, *vq = vb + (size_t)(r0 + rg) * rstride;
+    int row = r0 + rg;
 #pragma unroll 1
     for (int s = 0; s < kRing - 1 + n_steps; ++s) {
-      if (s < n_steps + kRing - 1) {
-        // prefetch step s (zero-filled past the segment); a group per step
-        const int row = r0 + s * RPW + rg;
+      {
+        // prefetch step s (zero-filled past the segment); one cp.async group per step
         const bool valid = s < n_steps && row < r1;
-        const size_t ro = (size_t)(valid ? row : r0) * rstride;
-        uint8_t *dst = ring + (s % kRing) * RG::kStepBytes;
+        const T *ks = valid ? kq : k_any, *vs = valid ? vq : v_any;
+        uint8_t *dst = ring + ((unsigned)s & (kRing - 1)) * RG::kStepBytes;
 #pragma unroll
         for (int j = 0; j < NCH; ++j) {
-          cp_async16(dst + j * 512, kb + ro + j * (LPR * EPC), valid);
-          cp_async16(dst + (NCH + j) * 512, vb + ro + j * (LPR * EPC), valid);
+          cp_async16(dst + j * 512, ks + j * (LPR * EPC), valid);
+          cp_async16(dst + (NCH + j) * 512, vs + j * (LPR * EPC), valid);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
+        kq += step_stride;
+        vq += step_stride;
+        row += RPW;
       }
       const int st = s - (kRing - 1);           // step consumed in this iteration
       if (st < 0) continue;
       asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
-      const uint8_t *src = ring + (st % kRing) * RG::kStepBytes;
+      const uint8_t *src = ring + ((unsigned)st & (kRing - 1)) * RG::kStepBytes;
       const bool valid = r0 + st * RPW + rg < r1;
       float kf[16];
 #pragma unroll
@@ -313,15 +318,16 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
             for (int i = 0; i < EPC; ++i)
               outp[g * D + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i] / l[g];
     } else {
-      float *pp = p.part + ((size_t)u * p.slots + (size_t)(gw - first)) * (size_t)(G * (D + 2));
+      constexpr int REC = rec_floats<D>();
+      float *pp = p.part + ((size_t)u * p.slots + (size_t)(gw - first)) * (size_t)(G * REC);
       if (rg == 0) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          if (sl == 0) { pp[g * (D + 2)] = m[g]; pp[g * (D + 2) + 1] = l[g]; }
+          if (sl == 0) { pp[g * REC] = m[g]; pp[g * REC + 1] = l[g]; }
 #pragma unroll
           for (int j = 0; j < NCH; ++j)
 #pragma unroll
-            for (int i = 0; i < EPC; ++i) pp[g * (D + 2) + 2 + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i];
+            for (int i = 0; i < EPC; ++i) pp[g * REC + 4 + j * (LPR * EPC) + sl * EPC + i] = acc[g][j * EPC + i];
         }
       }
       __threadfence();
@@ -332,19 +338,18 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
       if (last_in) {
         __threadfence();
         const int n_seg = (int)(last - first + 1);
-        const float *pu = p.part + (size_t)u * p.slots * (size_t)(G * (D + 2));
-        constexpr int kSeg = G * (D + 2);
-        // per-head maxima and normalisers, segments spread over the lanes
+        const float *pu = p.part + (size_t)u * p.slots * (size_t)(G * REC);
+        // segment weights: lane j holds segment j's (m, l) of every head
         float Mg[G], Lg[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           float mx = kNegInf;
-          for (int j = lane; j < n_seg; j += 32) mx = fmaxf(mx, __ldcg(pu + (size_t)j * kSeg + g * (D + 2)));
+          for (int j = lane; j < n_seg; j += 32) mx = fmaxf(mx, __ldcg(pu + ((size_t)j * G + g) * REC));
           Mg[g] = warp_max(mx);
           float ls = 0.f;
           for (int j = lane; j < n_seg; j += 32) {
-            const float mj = __ldcg(pu + (size_t)j * kSeg + g * (D + 2));
-            if (mj != kNegInf) ls += __ldcg(pu + (size_t)j * kSeg + g * (D + 2) + 1) * fast_exp2(mj - Mg[g]);
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(pu + ((size_t)j * G + g) * REC));
+            if (ml.x != kNegInf) ls += ml.y * fast_exp2(ml.x - Mg[g]);
           }
 #pragma unroll
           for (int o2 = 16; o2 > 0; o2 >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o2);
@@ -359,13 +364,19 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
           for (int i = 0; i < EPL; ++i) A[g][i] = 0.f;
 #pragma unroll 4
         for (int j = 0; j < n_seg; ++j) {
-          const float *q0 = pu + (size_t)j * kSeg;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float mj = __ldcg(q0 + g * (D + 2));
+            const float *rec = pu + ((size_t)j * G + g) * REC;
+            const float mj = __ldcg(rec);
             const float wgt = (mj == kNegInf) ? 0.f : fast_exp2(mj - Mg[g]);
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) A[g][i] = fmaf(__ldcg(q0 + g * (D + 2) + 2 + lane * EPL + i), wgt, A[g][i]);
+            if constexpr (EPL == 4) {
+              const float4 a4 = __ldcg(reinterpret_cast<const float4 *>(rec + 4) + lane);
+              A[g][0] = fmaf(a4.x, wgt, A[g][0]); A[g][1] = fmaf(a4.y, wgt, A[g][1]);
+              A[g][2] = fmaf(a4.z, wgt, A[g][2]); A[g][3] = fmaf(a4.w, wgt, A[g][3]);
+            } else {
+              const float2 a2 = __ldcg(reinterpret_cast<const float2 *>(rec + 4) + lane);
+              A[g][0] = fmaf(a2.x, wgt, A[g][0]); A[g][1] = fmaf(a2.y, wgt, A[g][1]);
+            }
           }
         }
 #pragma unroll
@@ -389,7 +400,7 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
 template <typename T, int D, int G>
 cudaError_t launch(const DecodeArgs &a, cudaStream_t st) {
   const int smem = DecRing<T>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(gqa_decode_streamk<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_limit((const void *)gqa_decode_streamk<T, D, G>, smem);
   if (e != cudaSuccess) return e;
   DecParams p;
   p.q = a.q; p.kc = a.k_c; p.vc = a.v_c; p.row_off = a.row_off; p.kv_len = a.kv_len; p.out = a.out;

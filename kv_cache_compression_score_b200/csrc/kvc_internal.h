@@ -68,3 +68,9 @@ cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
 int decode_slots(int max_kv_len);
 
 }  // namespace kvc
+
+namespace kvc {
+// Raise a kernel's dynamic shared-memory limit once per device (a host call
+// kept out of the per-launch path, so launches can be captured in graphs).
+cudaError_t ensure_smem_limit(const void *fn, int bytes);
+}  // namespace kvc

@@ -256,9 +256,9 @@ static cudaError_t launch_simt(const ScoreArgs &a, cudaStream_t st) {
   s.c = a.scale * kLog2e;
   const size_t smem = SimtSmem<T, D>::bytes(s.R_pad);
   cudaError_t e;
-  e = cudaFuncSetAttribute(score_stats_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_limit((const void *)score_stats_simt<T, D>, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(score_raw_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_limit((const void *)score_raw_simt<T, D>, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.n_kv, a.n_seqs);
   score_stats_simt<T, D><<<grid, kThreads, smem, st>>>(

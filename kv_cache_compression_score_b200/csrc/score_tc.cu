@@ -353,9 +353,9 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
   p.c = a.scale * kLog2e;
   const int smem = TcLayout<D>::kAlloc;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(score_tc_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, false>, smem)))
     return e;
-  if ((e = cudaFuncSetAttribute(score_tc_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
+  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, true>, smem)))
     return e;
   dim3 grid(a.n_chunks, a.n_kv, a.n_seqs);
   score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(p);
