@@ -174,6 +174,29 @@ kvc_status kvc_tsp_select_gather(kvc_dtype dt, int S, int n_rows, int w, int poo
                                  kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * kvc_tsp_select_gather_static: the same computation as
+ * kvc_tsp_select_gather, for callers that cannot allocate device memory for a
+ * workspace (code that must not touch the process' device allocator, e.g.
+ * running inside another component's memory pool or out-of-memory handler,
+ * or a serving loop that forbids allocations).  The pages have no
+ * counterpart: this is an interface convenience of the library.
+ *
+ * Scratch: a fixed array inside the library (1 MiB, every GPU that loads the
+ * library keeps it until the process exits).  S - w must not exceed 262,144;
+ * larger requests return KVC_ERR_UNSUPPORTED (use the workspace variant).
+ * The first call on a device resolves the array's device address for that
+ * device; make that first call before any stream capture.  All calls on one
+ * device share that device's array, which keeps the last call's contents:
+ * calls whose kernels can overlap on the GPU (for instance on different
+ * streams) race, so keep them on one stream or synchronise them.  Nothing in
+ * the array has to start at zero.  The call allocates and frees nothing.
+ * Other arguments, layouts and errors are those of kvc_tsp_select_gather.
+ * ------------------------------------------------------------------------ */
+kvc_status kvc_tsp_select_gather_static(kvc_dtype dt, int S, int n_rows, int w, int pool_k, int k_tsp,
+                                        const float *scores_raw, const void *hidden, int D,
+                                        int32_t *idx_out, void *hidden_out, kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * GQA decode attention over compact caches (decode reads the whole cache per
  * step: FastKV section 1; attention-variants page introduction):
  *   out[b][qh][:] = sum_{t < kv_len[b]} softmax_t(scale * q[b][qh] . Kc[o_b + t][h])

@@ -352,3 +352,71 @@ kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Token-selective propagation with library-owned scratch.
+//
+// For callers that cannot allocate device memory for a workspace -- code
+// running where the process' allocator must not be touched (inside another
+// library's memory pool or out-of-memory handler, or a latency-critical
+// serving loop that forbids allocation) -- this entry point keeps its only
+// scratch, the pooled head-summed scores of the prefix, in a fixed array
+// compiled into the library.  Every GPU that loads the library holds the
+// array (1 MiB) until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kStaticTspMaxPrefix = 262144;   // S - w limit of the static variant (floats)
+static __device__ __align__(256) float g_tsp_static_scratch[kStaticTspMaxPrefix];
+
+// Device address of the array on the current device, resolved once per
+// device (host code only sees a host-side stand-in under the array's name).
+kvc_status static_scratch(float **out) {
+  static std::mutex mu;
+  static std::vector<std::pair<int, float *>> resolved;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto &r : resolved)
+    if (r.first == dev) { *out = r.second; return KVC_OK; }
+  float *p = nullptr;
+  e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_tsp_static_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static TSP scratch");
+  resolved.push_back({dev, p});
+  *out = p;
+  return KVC_OK;
+}
+
+}  // namespace
+
+extern "C" kvc_status kvc_tsp_select_gather_static(kvc_dtype dt, int S, int n_rows, int w, int pool_k, int k_tsp,
+                                                   const float *scores_raw, const void *hidden, int D,
+                                                   int32_t *idx_out, void *hidden_out, kvc_stream_t stream) {
+  const int es = elem_size(dt);
+  if (!es) return fail(KVC_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+  if (S < 1 || w < 1 || w > S) return fail(KVC_ERR_INVALID_ARG, "need 1 <= w <= S (w=%d, S=%d)", w, S);
+  if (S - w > kStaticTspMaxPrefix)
+    return fail(KVC_ERR_UNSUPPORTED, "the static-scratch variant takes S - w <= %d (got %d); use "
+                "kvc_tsp_select_gather with a workspace", kStaticTspMaxPrefix, S - w);
+  if (n_rows < 1) return fail(KVC_ERR_INVALID_ARG, "n_rows must be >= 1");
+  if (pool_k < 1 || pool_k > 31 || pool_k % 2 == 0)
+    return fail(KVC_ERR_INVALID_ARG, "pool_k must be odd and in [1, 31] (got %d)", pool_k);
+  if (k_tsp < 0 || k_tsp > S - w) return fail(KVC_ERR_INVALID_ARG, "k_tsp must lie in [0, S - w] (got %d)", k_tsp);
+  if (D < 1 || ((int64_t)D * es) % 16 != 0)
+    return fail(KVC_ERR_UNSUPPORTED, "D * element size must be a positive multiple of 16 bytes");
+  if (!aligned16(scores_raw) || !aligned16(hidden) || !aligned16(idx_out) || !aligned16(hidden_out))
+    return fail(KVC_ERR_INVALID_ARG, "scores_raw, hidden, idx_out and hidden_out must be 16-byte aligned");
+  float *pooled = nullptr;
+  kvc_status s = static_scratch(&pooled);
+  if (s != KVC_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the pooled scores are fully rewritten before they are read: nothing to clear
+  cudaError_t e = kvc::tsp_pool(scores_raw, n_rows, S, w, pool_k, pooled, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tsp pool kernel");
+  e = kvc::tsp_select(pooled, S, w, k_tsp, idx_out, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tsp select kernel");
+  e = kvc::gather_hidden(hidden, hidden_out, idx_out, k_tsp + w, D * es, S, st);
+  if (e != cudaSuccess) return cuda_fail(e, "hidden gather kernel");
+  return KVC_OK;
+}

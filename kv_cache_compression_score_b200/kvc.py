@@ -36,6 +36,8 @@ SIGNATURES = {
     "kvc_tsp_workspace_size": (_c_sz, [_c_int, _c_int]),
     "kvc_tsp_select_gather": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p, _c_int, _c_p,
                                        _c_p, _c_p, _c_sz, _c_p]),
+    "kvc_tsp_select_gather_static": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p, _c_int,
+                                              _c_p, _c_p, _c_p]),
     "kvc_gqa_decode_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_i64, _c_p,
                                      _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
@@ -159,6 +161,15 @@ def kvc_tsp_select_gather(scores_raw, w: int, pool_k: int, k_tsp: int, hidden, i
     _check(lib().kvc_tsp_select_gather(dtype_code(hidden), S, n_rows, w, pool_k, k_tsp, _dptr(scores_raw),
                                        _dptr(hidden), hidden.shape[1], _dptr(idx_out), _dptr(hidden_out), _dptr(ws),
                                        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_tsp_select_gather_static(scores_raw, w: int, pool_k: int, k_tsp: int, hidden, idx_out, hidden_out,
+                                 stream=None) -> None:
+    """Token-selective propagation without a caller workspace (library-owned scratch)."""
+    n_rows, S = scores_raw.shape
+    _check(lib().kvc_tsp_select_gather_static(dtype_code(hidden), S, n_rows, w, pool_k, k_tsp, _dptr(scores_raw),
+                                              _dptr(hidden), hidden.shape[1], _dptr(idx_out), _dptr(hidden_out),
+                                              _stream(stream)))
 
 
 def kvc_gqa_decode_attn(q, k_c, v_c, kv_row_offset, kv_len, max_kv_len: int, scale: float, out, ws,
