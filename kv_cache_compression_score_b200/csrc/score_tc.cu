@@ -15,16 +15,23 @@
 //                over the rows, off_r = m_r + log2(l_r) merged from the
 //                stats partials.
 //
-// Warp roles (416 threads, one CTA per SM):
+// Warp roles (672 threads, one CTA per SM):
 //   warps 0-3   load K tiles (128 keys x d_h) with 16-byte cp.async straight
 //               into the 128-byte-swizzled K-major layout the MMA reads, a
-//               5-stage ring; 16-byte cp.async streams these strided head rows
-//               faster than tensor-map copies with 128-byte boxes.  Rows past
-//               the sequence are zero-filled (no read);
+//               5-stage ring.  Each loader thread's copies arrive on the
+//               stage's "full" barrier by themselves when they land
+//               (cp.async.mbarrier.arrive.noinc), so a loader only ever waits
+//               for a free stage.  Rows past the sequence are zero-filled
+//               (no read).  On this head-sliced pattern (256 B of every 2 KB
+//               key row) 16-byte cp.async streams as fast as tensor-map
+//               copies and leaves the ring fuller;
 //   warp 4      owns tensor memory (512 columns: four 128-column accumulators)
 //               and issues the MMAs from one thread;
-//   warps 5-12  epilogue: two warps per TMEM lane quarter, each reading half
-//               of the accumulator columns.
+//   warps 5-20  epilogue: four warps per TMEM lane quarter, each reading 32
+//               of the 128 accumulator columns, software-pipelined over
+//               16-column halves.
+// The grid runs the KV heads fastest, so the CTAs resident together read the
+// head slices of the same 2 KB key rows.
 // Every wait is bounded; a wait that gives up sets the device error word and
 // the CTA stops waiting (results are then flagged invalid, never a hang).
 #include "kvc_common.cuh"
@@ -36,14 +43,14 @@ namespace {
 constexpr int kBN = 128;          // keys per tile
 constexpr int kRows = 128;        // window-block rows (padded)
 constexpr int kStages = 5;        // K ring depth
-constexpr int kLag = kStages - 1; // tiles in flight per loader thread
 constexpr int kAccBufs = 4;       // TMEM accumulators
 constexpr int kLoadWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kEpiWarp0 = 5;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
+constexpr int kColBlocks = kEpiWarps / 4;   // 32-column blocks per lane quarter
 constexpr int kThreadsTC = (kLoadWarps + 1 + kEpiWarps) * 32;
-constexpr int kXch = 8;           // half-column exchange slots (score pass)
+constexpr int kXch = 8;           // column-block exchange slots (score pass)
 
 template <int D>
 struct TcLayout {
@@ -56,8 +63,10 @@ struct TcLayout {
   static constexpr int kBarCount = 2 * kStages + 2 * kAccBufs + 1 + kXch;
   static constexpr int kOffMisc = kOffBar + 256;
   static constexpr int kOffOff = kOffMisc + 16;              // off_r[128] (score pass)
-  static constexpr int kOffXch = kOffOff + kRows * 4;        // [kXch][128] (score) / m,l halves (stats)
-  static constexpr int kBytes = kOffXch + kXch * kBN * 4;
+  // score pass: [kXch][kColBlocks - 1][128] partial row sums; stats pass:
+  // m and l of every row for column blocks 1..kColBlocks-1
+  static constexpr int kOffXch = kOffOff + kRows * 4;
+  static constexpr int kBytes = kOffXch + kXch * (kColBlocks - 1) * kBN * 4;
   static constexpr int kAlloc = kBytes + 1024;               // room to align the base to 1 KB
   static_assert(kBarCount * 8 <= 256, "barrier area");
   static_assert(kOffOff % 16 == 0, "off[] is read as float4");
@@ -82,10 +91,15 @@ KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
                :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
 
+// arrive on *bar once every cp.async this thread issued so far has landed
+// (the arrival counts against the barrier's expected count)
+KVC_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
 // Q_win rows r = g * w + i of (b, h) into the 128-byte-swizzled K-major tile
 // with cp.async (all chunks in flight at once); rows >= R are zero-filled.
-// Completion, publication to the tensor core and the q_full arrive are done
-// by the caller together with its first K tiles.
+// The caller makes their completion arrive on q_full.
 template <int D>
 KVC_DEVINL void stage_q_async(uint8_t *sq, const TcParams &p, int b, int h, int tid, int nthreads) {
   constexpr int kChunks = D / 8;   // 16-byte chunks per row
@@ -100,62 +114,74 @@ KVC_DEVINL void stage_q_async(uint8_t *sq, const TcParams &p, int b, int h, int 
   }
 }
 
-// Stats-pass reduction of 32 logits of one window row (keys k0..k0+31):
-// online max / sum of 2^(c*z - m); masked keys (beyond the chunk end or the
-// row's causal limit) contribute nothing.
-KVC_DEVINL void epi_stats_chunk(float *v, int k0, int key_end, int P, int row_pos, float c, float &m, float &l) {
-  if (!(k0 + 31 <= P && k0 + 32 <= key_end)) {
+constexpr float kSlack = 8.f;   // stats pass: log2 headroom before the running max moves
+
+// Stats-pass reduction of 16 logits of one window row (keys k0..k0+15):
+// running sum of 2^(c*z - m).  The reference m only moves, by warp vote, when
+// a logit exceeds it by more than kSlack (so every term stays <= 2^kSlack and
+// the rescale of l is rare and warp-uniform).  Masked keys (beyond the chunk
+// end or the row's causal limit) contribute nothing.
+KVC_DEVINL void epi_stats16(uint32_t (&r)[16], int k0, int key_end, int P, int row_pos, float c, float &m, float &l) {
+  float v[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+  if (!(k0 + 15 <= P && k0 + 16 <= key_end)) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
       const int key = k0 + j;
       if (!(key < key_end && key <= row_pos)) v[j] = kNegInf;
     }
   }
-  float t[16];
+  float t[8];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) t[j] = fmaxf(v[j], v[j + 16]);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) t[j] = fmaxf(t[j], t[j + 8]);
+  for (int j = 0; j < 8; ++j) t[j] = fmaxf(v[j], v[j + 8]);
 #pragma unroll
   for (int j = 0; j < 4; ++j) t[j] = fmaxf(t[j], t[j + 4]);
   const float cmax = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])) * c;   // c > 0
-  const float mn = fmaxf(m, cmax);
-  const float ms = (mn == kNegInf) ? 0.f : mn;
-  float a[8];
+  const bool need = cmax > m + kSlack;
+  if (__any_sync(0xffffffffu, need)) {
+    const float mn = need ? cmax : m;
+    if (need) l *= (m == kNegInf) ? 0.f : fast_exp2(m - mn);
+    m = mn;
+  }
+  const float ms = (m == kNegInf) ? 0.f : m;
+  float a[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) a[j] = fast_exp2(fmaf(v[j], c, -ms));
+  for (int j = 0; j < 4; ++j) a[j] = fast_exp2(fmaf(v[j], c, -ms));
 #pragma unroll
-  for (int j = 8; j < 32; ++j) a[j & 7] += fast_exp2(fmaf(v[j], c, -ms));
-  const float cs = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
-  l = fmaf(l, fast_exp2(m - ms), cs);
-  m = mn;
+  for (int j = 4; j < 16; ++j) a[j & 3] += fast_exp2(fmaf(v[j], c, -ms));
+  l += (a[0] + a[1]) + (a[2] + a[3]);
 }
 
-// Score-pass accumulation for one key over window rows r0..r0+31:
-// acc += 2^(c*z_r - off_r); rows above the key's causal limit are skipped.
-KVC_DEVINL void epi_score_chunk(const float *v, const float *off, int r0, int key, int P, const TcParams &p,
-                                float *acc8) {
+// Score-pass accumulation for one key over window rows r0..r0+15:
+// returns the sum of 2^(c*z_r - off_r); rows above the key's causal limit are
+// skipped.
+KVC_DEVINL float epi_score16(uint32_t (&rr)[16], const float *off, int r0, int key, int P, const TcParams &p) {
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
   if (key <= P) {     // prefix key (or the first window key): visible to every row
 #pragma unroll
-    for (int r = 0; r < 32; r += 4) {
+    for (int r = 0; r < 16; r += 4) {
       const float4 o4 = *reinterpret_cast<const float4 *>(off + r0 + r);
-      acc8[(r >> 2) & 7] += (fast_exp2(fmaf(v[r], p.c, -o4.x)) + fast_exp2(fmaf(v[r + 1], p.c, -o4.y))) +
-                            (fast_exp2(fmaf(v[r + 2], p.c, -o4.z)) + fast_exp2(fmaf(v[r + 3], p.c, -o4.w)));
+      a[(r >> 2) & 3] += (fast_exp2(fmaf(__uint_as_float(rr[r]), p.c, -o4.x)) +
+                          fast_exp2(fmaf(__uint_as_float(rr[r + 1]), p.c, -o4.y))) +
+                         (fast_exp2(fmaf(__uint_as_float(rr[r + 2]), p.c, -o4.z)) +
+                          fast_exp2(fmaf(__uint_as_float(rr[r + 3]), p.c, -o4.w)));
     }
   } else {            // window key: row r (window row r % w) sees it when key <= P + r % w
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
+    for (int r = 0; r < 16; ++r) {
       const int row = r0 + r;
-      if (row < p.R && key <= P + row % p.w) acc8[r & 7] += fast_exp2(fmaf(v[r], p.c, -off[row]));
+      if (row < p.R && key <= P + row % p.w) a[r & 3] += fast_exp2(fmaf(__uint_as_float(rr[r]), p.c, -off[row]));
     }
   }
+  return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 template <int D, bool kScorePass>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 score_tc_kernel(TcParams p) {
   using L = TcLayout<D>;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
   const int t0 = p.cu_seqlens[b], len = p.cu_seqlens[b + 1] - t0;
   const int key_begin = c * p.keys_per_chunk;
   if (key_begin >= len) return;
@@ -182,7 +208,7 @@ score_tc_kernel(TcParams p) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], kLoadWarps * 32); mbar_init(&empty[s], 1); }
     for (int s = 0; s < kAccBufs; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
     mbar_init(q_full, kLoadWarps * 32);
-    for (int s = 0; s < kXch; ++s) mbar_init(&xch_full[s], 4);
+    for (int s = 0; s < kXch; ++s) mbar_init(&xch_full[s], 4 * (kColBlocks - 1));
     *cta_err = 0;
     fence_mbar_init();
   }
@@ -196,35 +222,25 @@ score_tc_kernel(TcParams p) {
     // ------------------------------------------------------------ K loaders
     const int lt = threadIdx.x;                      // 0..127
     stage_q_async<D>(sq, p, b, h, lt, kLoadWarps * 32);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    bool q_published = false;
+    cp_async_arrive_noinc(q_full);
     constexpr int kChunks = kBN * D / 8;             // 16-byte chunks per tile
     const uint8_t *kbase = reinterpret_cast<const uint8_t *>(p.k);
-    for (int t = 0; t < n_tiles + kLag; ++t) {
-      if (t < n_tiles) {
-        const int s = t % kStages;
-        if (!*cta_err && !mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1)) *cta_err = 1;
-        const int key0 = key_begin + t * kBN;
-        uint8_t *dst = sk + s * L::kKBytes;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t % kStages;
+      if (!*cta_err && !mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1)) *cta_err = 1;
+      const int key0 = key_begin + t * kBN;
+      uint8_t *dst = sk + s * L::kKBytes;
 #pragma unroll 4
-        for (int e = lt; e < kChunks; e += kLoadWarps * 32) {
-          const int row = e / (D / 8), ch = e % (D / 8);
-          const int atom = ch >> 3, c16 = ch & 7;
-          const bool valid = key0 + row < key_end;
-          const uint8_t *src = kbase + ((size_t)(t0 + (valid ? key0 + row : 0)) * p.n_kv + h) * (D * 2) + ch * 16;
-          cp_async16(dst + atom * L::kAtomBytes + row * 128 + ((c16 ^ (row & 7)) << 4), src, valid);
-        }
+      for (int e = lt; e < kChunks; e += kLoadWarps * 32) {
+        const int row = e / (D / 8), ch = e % (D / 8);
+        const int atom = ch >> 3, c16 = ch & 7;
+        const bool valid = key0 + row < key_end;
+        const uint8_t *src = kbase + ((size_t)(t0 + (valid ? key0 + row : 0)) * p.n_kv + h) * (D * 2) + ch * 16;
+        cp_async16(dst + atom * L::kAtomBytes + row * 128 + ((c16 ^ (row & 7)) << 4), src, valid);
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
-      if (t >= kLag) {
-        // the window block (group 0) and tile t - kLag have landed for this
-        // thread: publish them to the tensor core
-        asm volatile("cp.async.wait_group %0;" :: "n"(kLag) : "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (!q_published) { mbar_arrive(q_full); q_published = true; }
-        mbar_arrive(&full[(t - kLag) % kStages]);
-      }
+      cp_async_arrive_noinc(&full[s]);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -236,6 +252,9 @@ score_tc_kernel(TcParams p) {
         const int s = t % kStages, buf = t % kAccBufs;
         if (!mbar_wait(&full[s], (t / kStages) & 1)) { *cta_err = 1; break; }
         if (!mbar_wait(&acc_empty[buf], ((t / kAccBufs) & 1) ^ 1)) { *cta_err = 1; break; }
+        // the stage was written through the generic proxy (cp.async); order
+        // those writes, now visible to this thread, before the tensor core's reads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * 128;
 #pragma unroll
@@ -255,10 +274,10 @@ score_tc_kernel(TcParams p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - kEpiWarp0;                 // 0..7
-    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..255
+    const int ew = warp - kEpiWarp0;                 // 0..15
+    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..511
     const int quarter = warp & 3;                    // TMEM lanes this warp may access
-    const int half = ew >> 2;                        // which 64 accumulator columns
+    const int cb = ew >> 2;                          // which 32 accumulator columns
     const int my_lane = 32 * quarter + lane;         // row (stats) or key (score)
     if (kScorePass) {
       // merge the stats partials of every row into off_r = M + log2(L)
@@ -283,51 +302,71 @@ score_tc_kernel(TcParams p) {
 
     float m = kNegInf, l = 0.f;
     const int row_pos = P + (my_lane % max(p.w, 1));   // stats pass: this thread's row position
-    for (int t = 0; t < n_tiles; ++t) {
-      const int buf = t % kAccBufs;
-      const bool got = *cta_err ? true : mbar_wait(&acc_full[buf], (t / kAccBufs) & 1);
+    const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16) + cb * 32;
+    auto wait_full = [&](int t) {
+      const bool got = *cta_err ? true : mbar_wait(&acc_full[t % kAccBufs], (t / kAccBufs) & 1);
       if (!__all_sync(0xffffffffu, got) && lane == 0) *cta_err = 1;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * 128 + half * 64;
+    };
+    // software pipeline over 16-column halves: the TMEM load of the next half
+    // is in flight while the current one is reduced
+    uint32_t ra[16], rb[16];
+    if (n_tiles > 0) {
+      wait_full(0);
+      tmem_ld16(t_lane, ra);
+      tmem_wait_ld16(ra);
+    }
+    for (int t = 0; t < n_tiles; ++t) {
+      const int buf = t % kAccBufs;
       const int key0 = key_begin + t * kBN;
-      float va[32], vb[32];
-      float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      tmem_ld32(taddr, va);
-      tmem_wait_ld();
-      tmem_ld32(taddr + 32, vb);
-      if (!kScorePass) epi_stats_chunk(va, key0 + half * 64, key_end, P, row_pos, p.c, m, l);
-      else epi_score_chunk(va, off, half * 64, key0 + my_lane, P, p, acc8);
-      tmem_wait_ld();
+      tmem_ld16(t_lane + buf * 128 + 16, rb);
+      float sum = 0.f;
+      if (!kScorePass) epi_stats16(ra, key0 + cb * 32, key_end, P, row_pos, p.c, m, l);
+      else sum = epi_score16(ra, off, cb * 32, key0 + my_lane, P, p);
+      tmem_wait_ld16(rb);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);    // this warp's columns are read
-      if (!kScorePass) epi_stats_chunk(vb, key0 + half * 64 + 32, key_end, P, row_pos, p.c, m, l);
-      else epi_score_chunk(vb, off, half * 64 + 32, key0 + my_lane, P, p, acc8);
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);    // this warp's columns of tile t are read
+      if (t + 1 < n_tiles) {
+        wait_full(t + 1);
+        tmem_ld16(t_lane + ((t + 1) % kAccBufs) * 128, ra);
+      }
+      if (!kScorePass) epi_stats16(rb, key0 + cb * 32 + 16, key_end, P, row_pos, p.c, m, l);
+      else sum += epi_score16(rb, off, cb * 32 + 16, key0 + my_lane, P, p);
       if (kScorePass) {
-        const float sum = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
         const int slot = t % kXch;
+        float *xs = xch + (size_t)slot * (kColBlocks - 1) * kBN;
         const int key = key0 + my_lane;
-        if (half == 1) {
-          xch[slot * kBN + my_lane] = sum;
+        if (cb > 0) {
+          xs[(cb - 1) * kBN + my_lane] = sum;
           __syncwarp();
           if (lane == 0) mbar_arrive(&xch_full[slot]);
         } else {
           const bool ok = *cta_err ? true : mbar_wait(&xch_full[slot], (t / kXch) & 1);
           if (!__all_sync(0xffffffffu, ok) && lane == 0) *cta_err = 1;
-          if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = sum + xch[slot * kBN + my_lane];
+          float tot = sum;
+#pragma unroll
+          for (int j = 0; j < kColBlocks - 1; ++j) tot += xs[j * kBN + my_lane];
+          if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = tot;
         }
       }
+      if (t + 1 < n_tiles) tmem_wait_ld16(ra);
     }
     if (!kScorePass) {
-      // merge the two column halves of every row, then publish the partial
-      float *xm = xch, *xl = xch + kRows;
-      if (half == 1) { xm[my_lane] = m; xl[my_lane] = l; }
+      // merge the column blocks of every row, then publish the partial
+      float *xm = xch, *xl = xch + (kColBlocks - 1) * kRows;
+      if (cb > 0) { xm[(cb - 1) * kRows + my_lane] = m; xl[(cb - 1) * kRows + my_lane] = l; }
       asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
-      if (half == 0 && my_lane < p.R) {
-        const float m2 = xm[my_lane], l2 = xl[my_lane];
-        const float mn = fmaxf(m, m2);
+      if (cb == 0 && my_lane < p.R) {
+        float mn = m;
+#pragma unroll
+        for (int j = 0; j < kColBlocks - 1; ++j) mn = fmaxf(mn, xm[j * kRows + my_lane]);
         float ls = 0.f;
-        if (mn != kNegInf) ls = l * fast_exp2(m - mn) + l2 * fast_exp2(m2 - mn);
+        if (mn != kNegInf) {
+          ls = l * fast_exp2(m - mn);
+#pragma unroll
+          for (int j = 0; j < kColBlocks - 1; ++j) ls += xl[j * kRows + my_lane] * fast_exp2(xm[j * kRows + my_lane] - mn);
+        }
         p.part[((size_t)(b * p.n_kv + h) * p.n_chunks + c) * kRows + my_lane] = make_float2(mn, ls);
       }
     }
@@ -357,7 +396,7 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
     return e;
   if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, true>, smem)))
     return e;
-  dim3 grid(a.n_chunks, a.n_kv, a.n_seqs);
+  dim3 grid(a.n_kv, a.n_chunks, a.n_seqs);
   score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(p);
   if ((e = cudaGetLastError())) return e;
   score_tc_kernel<D, true><<<grid, kThreadsTC, smem, st>>>(p);
