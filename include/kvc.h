@@ -29,9 +29,13 @@
  *     call only.
  *   - Scratch memory is a caller-provided device workspace whose size comes
  *     from the matching *_workspace_size() query; it may be reused between
- *     calls on the same stream.  The decode workspace holds completion
- *     counters that must be zero before its first use (cudaMemset to 0 once);
- *     every decode call leaves them zero again.
+ *     calls on the same stream.  The score and decode workspaces hold
+ *     counters that must be zero before their first use (cudaMemset to 0
+ *     once); every call leaves them zero again.  The first int32 of every
+ *     workspace is a device error word: a kernel whose bounded wait gave up
+ *     (a pipeline or another CTA did not answer in time) sets it nonzero and
+ *     stops waiting instead of hanging; that call's results are invalid.
+ *     After such a call, zero the workspace again before reusing it.
  *   - Ragged batches: n_seqs sequences packed along the token axis; seqlens_host
  *     (host int32[n_seqs]) gives the lengths, cu_seqlens (device int32[n_seqs+1])
  *     their prefix sums starting at 0.  Both must describe the same batch.
@@ -113,7 +117,11 @@ int64_t kvc_budget_offsets(int n_seqs, const int32_t *seqlens_host, int budget,
  * G = n_h / n_kv; the window block has G * w <= 256 rows (and a multiple of 16
  * rows for KVC_BF16).  pool_k odd in [1, 31].  scores_raw may be NULL.
  * q_win: [n_seqs * w, n_h, d_h];  k: [T, n_kv, d_h];  scores, scores_raw:
- * float32 [n_kv, T].  ws: kvc_score_window_workspace_size() bytes.
+ * float32 [n_kv, T].  ws: kvc_score_window_workspace_size() bytes, zeroed
+ * before its first use (it holds per-(sequence, head) arrival counters).
+ * When every (sequence, head, key chunk) work item fits on the GPU at once,
+ * KVC_BF16 scoring runs as one cooperative launch (both passes and the pool);
+ * otherwise as three launches.  Results are the same either way.
  * ------------------------------------------------------------------------ */
 size_t kvc_score_window_workspace_size(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host,
                                        int n_h, int n_kv, int d_h, int w);

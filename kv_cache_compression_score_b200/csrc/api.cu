@@ -64,10 +64,10 @@ kvc_status check_batch(int n_seqs, const int32_t *seqlens_host, int min_each, Ba
 
 // --------------------------------------------------------- scoring plan
 struct ScorePlan {
-  bool tc = false;
+  bool tc = false, fused = false;
   int R = 0, R_pad = 0, tile = 0, keys_per_chunk = 0, n_chunks = 0;
   Batch bt;
-  size_t off_part = 0, off_raw = 0, bytes = 0;
+  size_t off_sync = 0, off_part = 0, off_raw = 0, bytes = 0;
 };
 
 kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w,
@@ -105,7 +105,10 @@ kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int
   tpc = std::max(1, std::min(tpc, std::max(1, max_tiles)));
   pl->keys_per_chunk = tpc * pl->tile;
   pl->n_chunks = std::max(1, (pl->bt.max_len + pl->keys_per_chunk - 1) / pl->keys_per_chunk);
-  pl->off_part = kErrWordBytes;
+  // one cooperative launch when the whole grid is resident at once (one CTA per SM)
+  pl->fused = pl->tc && (int64_t)n_kv * pl->n_chunks * n_seqs <= kvc::kNumSMs;
+  pl->off_sync = kErrWordBytes;
+  pl->off_part = round_up(pl->off_sync + (size_t)n_seqs * n_kv * 4 * sizeof(int), 256);
   const size_t part_bytes = (size_t)n_seqs * n_kv * pl->n_chunks * pl->R_pad * sizeof(float2);
   pl->off_raw = round_up(pl->off_part + part_bytes, 256);
   pl->bytes = pl->off_raw + round_up((size_t)n_kv * pl->bt.T * sizeof(float), 256);
@@ -223,12 +226,17 @@ kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_hos
   a.part = reinterpret_cast<float2 *>(wsb + pl.off_part);
   a.raw = scores_raw ? scores_raw : reinterpret_cast<float *>(wsb + pl.off_raw);
   a.err = reinterpret_cast<int *>(wsb);
+  a.sync = reinterpret_cast<int *>(wsb + pl.off_sync);
+  a.scores = scores;
+  a.pool_k = pool_k;
+  a.fused = pl.fused;
   a.T_total = (int)pl.bt.T;
   a.n_chunks = pl.n_chunks;
   a.keys_per_chunk = pl.keys_per_chunk;
   a.R_pad = pl.R_pad;
   cudaError_t e = pl.tc ? kvc::score_window_tc(a, st) : kvc::score_window_simt(a, st);
   if (e != cudaSuccess) return cuda_fail(e, "score kernels");
+  if (pl.fused) return KVC_OK;   // the pool ran inside the fused launch
   e = kvc::pool_prefix(a.raw, scores, cu_seqlens, n_seqs, n_kv, a.T_total, pl.bt.max_len, w, pool_k, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   return KVC_OK;

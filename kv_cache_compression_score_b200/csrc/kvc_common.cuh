@@ -66,10 +66,18 @@ KVC_DEVINL uint32_t smem_u32(const void *p) {
 
 // ---------------------------------------------------------------------------
 // mbarrier (shared-memory transaction barrier) with bounded waits.  A wait
-// that runs out of iterations records an error code and returns false; the
-// caller then stops issuing work and leaves through its normal exit path.
+// that runs past its time limit returns false; the caller records an error
+// code, stops issuing work and leaves through its normal exit path.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kSpinLimit = 1u << 22;   // a few seconds at most; healthy waits take microseconds
+constexpr uint32_t kSpinLimit = 1u << 22;          // iteration bound of plain polling loops
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s; healthy waits take microseconds
+constexpr uint32_t kSuspendHintNs = 1000000;       // a try_wait may sleep up to this long
+
+KVC_DEVINL uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 KVC_DEVINL void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
@@ -85,19 +93,24 @@ KVC_DEVINL void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
                :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
+// One wait step: the thread sleeps in hardware until the phase with the given
+// parity completes (returns true) or the suspend hint runs out (false), so a
+// waiting warp takes no issue slots from the warps doing the work.
 KVC_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile("{\n\t.reg .pred p;\n\t"
-               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
                "selp.u32 %0, 1, 0, p;\n\t}"
-               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
   return ok != 0;
 }
-// Returns false when the wait gave up (after kSpinLimit polls).
+// Returns false when the wait gave up (after kWaitLimitNs).
 KVC_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  return true;
 }
 
 // ---------------------------------------------------------------------------

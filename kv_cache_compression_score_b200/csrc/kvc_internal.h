@@ -21,7 +21,11 @@ struct ScoreArgs {
   const void *k;
   float2 *part;          // [n_seqs, n_kv, n_chunks, R_pad] (m, l) per window row
   float *raw;            // [n_kv, T_total]
+  float *scores;         // [n_kv, T_total] pooled (written by the fused path)
+  int *sync;             // fused path: 4 counters per (sequence, KV head), zero between calls
   int *err;              // device error word (nonzero: a bounded wait gave up)
+  int pool_k;
+  bool fused;            // both passes and the pool in one cooperative launch
   int T_total;
   int n_chunks;          // key chunks per (sequence, KV head) in the launch grid
   int keys_per_chunk;    // multiple of the kernel's key tile

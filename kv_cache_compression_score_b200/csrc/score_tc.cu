@@ -32,6 +32,17 @@
 //               16-column halves.
 // The grid runs the KV heads fastest, so the CTAs resident together read the
 // head slices of the same 2 KB key rows.
+//
+// When the whole grid fits on the GPU at once (one CTA per SM), both passes
+// and the max-pool run in ONE cooperative launch: a CTA publishes its stats
+// partial, waits on a per-(sequence, head) arrival counter for the other key
+// chunks of its head, then runs the score pass over its own chunk in reverse
+// tile order -- the last kStages tiles of the stats pass are still in its
+// shared-memory ring and are not loaded again, the rest mostly come from L2 --
+// and after a second counter pools its chunk (halo from the neighbours' raw
+// scores).  This saves a launch, the window-block staging, the tensor-memory
+// allocation and the separate pool kernel, and a third of the second K pass.
+// Otherwise the two passes are separate launches and the pool kernel follows.
 // Every wait is bounded; a wait that gives up sets the device error word and
 // the CTA stops waiting (results are then flagged invalid, never a hang).
 #include "kvc_common.cuh"
@@ -80,9 +91,25 @@ struct TcParams {
   const int *cu_seqlens;
   float2 *part;
   float *raw;
+  float *scores;   // fused path: pooled output
+  int *sync;       // fused path: 4 counters per (sequence, KV head), zero between calls
   int *err;
-  int n_h, n_kv, G, w, R, n_chunks, keys_per_chunk, T_total;
+  int n_h, n_kv, G, w, R, n_chunks, keys_per_chunk, T_total, pool_r;
   float c;   // scale * log2(e)
+};
+
+// Shared-memory objects of one CTA.
+struct TcSmem {
+  uint8_t *sq, *sk;
+  uint64_t *full, *empty, *acc_full, *acc_empty, *q_full, *xch_full;
+  uint32_t *tmem_slot;
+  volatile int *cta_err;
+  float *off, *xch;
+};
+
+// The CTA's share of the work: key chunk c of KV head h of sequence b.
+struct TcWork {
+  int b, h, c, t0, len, P, key_begin, key_end, n_tiles;
 };
 
 // 16-byte cp.async, zero-filled (no global read) when !valid
@@ -177,81 +204,108 @@ KVC_DEVINL float epi_score16(uint32_t (&rr)[16], const float *off, int r0, int k
   return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
-template <int D, bool kScorePass>
-__global__ void __launch_bounds__(kThreadsTC, 1)
-score_tc_kernel(TcParams p) {
+template <int D>
+KVC_DEVINL TcSmem carve_smem(uint8_t *smem_raw) {
   using L = TcLayout<D>;
-  const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
-  const int t0 = p.cu_seqlens[b], len = p.cu_seqlens[b + 1] - t0;
-  const int key_begin = c * p.keys_per_chunk;
-  if (key_begin >= len) return;
-  const int key_end = min(len, key_begin + p.keys_per_chunk);
-  const int n_tiles = (key_end - key_begin + kBN - 1) / kBN;
-  const int P = len - p.w;
-
-  extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sq = smem + L::kOffQ;
-  uint8_t *sk = smem + L::kOffK;
+  TcSmem sm;
+  sm.sq = smem + L::kOffQ;
+  sm.sk = smem + L::kOffK;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
-  uint64_t *full = bars, *empty = bars + kStages;
-  uint64_t *acc_full = bars + 2 * kStages, *acc_empty = acc_full + kAccBufs;
-  uint64_t *q_full = acc_empty + kAccBufs;
-  uint64_t *xch_full = q_full + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
-  volatile int *cta_err = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
-  float *off = reinterpret_cast<float *>(smem + L::kOffOff);
-  float *xch = reinterpret_cast<float *>(smem + L::kOffXch);
+  sm.full = bars;
+  sm.empty = bars + kStages;
+  sm.acc_full = bars + 2 * kStages;
+  sm.acc_empty = sm.acc_full + kAccBufs;
+  sm.q_full = sm.acc_empty + kAccBufs;
+  sm.xch_full = sm.q_full + 1;
+  sm.tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+  sm.cta_err = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
+  sm.off = reinterpret_cast<float *>(smem + L::kOffOff);
+  sm.xch = reinterpret_cast<float *>(smem + L::kOffXch);
+  return sm;
+}
 
-  const int warp = warp_id(), lane = lane_id();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], kLoadWarps * 32); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < kAccBufs; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
-    mbar_init(q_full, kLoadWarps * 32);
-    for (int s = 0; s < kXch; ++s) mbar_init(&xch_full[s], 4 * (kColBlocks - 1));
-    *cta_err = 0;
-    fence_mbar_init();
+// (Re)initialise the pipeline barriers (one thread; the caller fences and syncs).
+KVC_DEVINL void init_pass_barriers(const TcSmem &sm, bool reinit) {
+  auto init = [&](uint64_t *bar, uint32_t count) {
+    if (reinit) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
+    mbar_init(bar, count);
+  };
+  for (int s = 0; s < kStages; ++s) { init(&sm.full[s], kLoadWarps * 32); init(&sm.empty[s], 1); }
+  for (int s = 0; s < kAccBufs; ++s) { init(&sm.acc_full[s], 1); init(&sm.acc_empty[s], kEpiWarps); }
+  for (int s = 0; s < kXch; ++s) init(&sm.xch_full[s], 4 * (kColBlocks - 1));
+}
+
+KVC_DEVINL int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One thread: announce this CTA on *ctr, then wait (bounded) until n CTAs did.
+KVC_DEVINL bool arrive_and_wait(int *ctr, int n) {
+  __threadfence();
+  atomicAdd(ctr, 1);
+  const uint64_t t0 = global_ns();
+  while (ld_acquire(ctr) < n) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
   }
-  if (warp == kMmaWarp) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  return true;
+}
 
+// One pass over the CTA's key chunk, all warp roles.
+//   kScorePass = false: stats pass, writes the (m, l) partial of every row.
+//   kScorePass = true:  score pass, writes the raw scores of the chunk; off[]
+//                       must hold off_r.  With rev, tiles run last to first
+//                       and the last min(kStages, n_tiles) tiles are taken as
+//                       already resident in the ring (left by the stats pass).
+template <int D, bool kScorePass>
+KVC_DEVINL void tc_pass(const TcParams &p, const TcSmem &sm, const TcWork &wk, uint32_t tmem_base, bool rev) {
+  using L = TcLayout<D>;
+  const int warp = warp_id(), lane = lane_id();
+  const int n = wk.n_tiles;
+  const int resident = rev ? min(kStages, n) : 0;
+  auto tile_of = [&](int j) { return rev ? n - 1 - j : j; };
   if (warp < kLoadWarps) {
     // ------------------------------------------------------------ K loaders
     const int lt = threadIdx.x;                      // 0..127
-    stage_q_async<D>(sq, p, b, h, lt, kLoadWarps * 32);
-    cp_async_arrive_noinc(q_full);
     constexpr int kChunks = kBN * D / 8;             // 16-byte chunks per tile
     const uint8_t *kbase = reinterpret_cast<const uint8_t *>(p.k);
-    for (int t = 0; t < n_tiles; ++t) {
-      const int s = t % kStages;
-      if (!*cta_err && !mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1)) *cta_err = 1;
-      const int key0 = key_begin + t * kBN;
-      uint8_t *dst = sk + s * L::kKBytes;
+    for (int j = resident; j < n; ++j) {
+      const int t = tile_of(j), s = t % kStages;
+      // use u of slot s in this pass (in rev mode use 0 is the resident
+      // tile): wait until the MMA of use u - 1 released the slot, i.e. for
+      // phase u - 1 of its "empty" barrier (u = 0: nothing to wait for)
+      const int u = j / kStages;
+      if (!*sm.cta_err && !mbar_wait(&sm.empty[s], (u - 1) & 1)) *sm.cta_err = 1;
+      const int key0 = wk.key_begin + t * kBN;
+      uint8_t *dst = sm.sk + s * L::kKBytes;
 #pragma unroll 4
       for (int e = lt; e < kChunks; e += kLoadWarps * 32) {
         const int row = e / (D / 8), ch = e % (D / 8);
         const int atom = ch >> 3, c16 = ch & 7;
-        const bool valid = key0 + row < key_end;
-        const uint8_t *src = kbase + ((size_t)(t0 + (valid ? key0 + row : 0)) * p.n_kv + h) * (D * 2) + ch * 16;
+        const bool valid = key0 + row < wk.key_end;
+        const uint8_t *src = kbase + ((size_t)(wk.t0 + (valid ? key0 + row : 0)) * p.n_kv + wk.h) * (D * 2) + ch * 16;
         cp_async16(dst + atom * L::kAtomBytes + row * 128 + ((c16 ^ (row & 7)) << 4), src, valid);
       }
-      cp_async_arrive_noinc(&full[s]);
+      cp_async_arrive_noinc(&sm.full[s]);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-      const uint32_t q_addr = smem_u32(sq), k_addr = smem_u32(sk);
-      if (!mbar_wait(q_full, 0)) *cta_err = 1;
+      const uint32_t q_addr = smem_u32(sm.sq), k_addr = smem_u32(sm.sk);
       int issued = 0;
-      for (int t = 0; t < n_tiles && !*cta_err; ++t) {
-        const int s = t % kStages, buf = t % kAccBufs;
-        if (!mbar_wait(&full[s], (t / kStages) & 1)) { *cta_err = 1; break; }
-        if (!mbar_wait(&acc_empty[buf], ((t / kAccBufs) & 1) ^ 1)) { *cta_err = 1; break; }
+      for (int j = 0; j < n && !*sm.cta_err; ++j) {
+        const int t = tile_of(j), s = t % kStages, buf = j % kAccBufs;
+        const int u = j / kStages;
+        if (j >= resident) {
+          const int load_no = rev ? u - 1 : u;
+          if (!mbar_wait(&sm.full[s], load_no & 1)) { *sm.cta_err = 1; break; }
+        }
+        if (!mbar_wait(&sm.acc_empty[buf], ((j / kAccBufs) & 1) ^ 1)) { *sm.cta_err = 1; break; }
         // the stage was written through the generic proxy (cp.async); order
         // those writes, now visible to this thread, before the tensor core's reads
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -265,117 +319,239 @@ score_tc_kernel(TcParams p) {
           if (kScorePass) umma_bf16(d_tmem, dk, dq, idesc, ks > 0);
           else umma_bf16(d_tmem, dq, dk, idesc, ks > 0);
         }
-        umma_commit(&empty[s]);
-        umma_commit(&acc_full[buf]);
-        issued = t + 1;
+        // free the stage only if a later load of this pass waits for it
+        if (j + kStages < n) umma_commit(&sm.empty[s]);
+        umma_commit(&sm.acc_full[buf]);
+        issued = j + 1;
       }
       // drain: the last commit tracks every MMA issued by this thread
-      if (issued > 0 && !mbar_wait(&acc_full[(issued - 1) % kAccBufs], ((issued - 1) / kAccBufs) & 1)) *cta_err = 1;
+      if (issued > 0 && !mbar_wait(&sm.acc_full[(issued - 1) % kAccBufs], ((issued - 1) / kAccBufs) & 1))
+        *sm.cta_err = 1;
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - kEpiWarp0;                 // 0..15
-    const int et = threadIdx.x - kEpiWarp0 * 32;     // 0..511
     const int quarter = warp & 3;                    // TMEM lanes this warp may access
     const int cb = ew >> 2;                          // which 32 accumulator columns
     const int my_lane = 32 * quarter + lane;         // row (stats) or key (score)
-    if (kScorePass) {
-      // merge the stats partials of every row into off_r = M + log2(L)
-      const float2 *pp = p.part + (size_t)(b * p.n_kv + h) * p.n_chunks * kRows;
-      const int nc = (len + p.keys_per_chunk - 1) / p.keys_per_chunk;
-      for (int r = et; r < kRows; r += kEpiWarps * 32) {
-        float o = kPosInf;
-        if (r < p.R) {
-          float M = kNegInf;
-          for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, pp[(size_t)cc * kRows + r].x);
-          float Ls = 0.f;
-          for (int cc = 0; cc < nc; ++cc) {
-            const float2 v = pp[(size_t)cc * kRows + r];
-            if (v.x != kNegInf) Ls += v.y * fast_exp2(v.x - M);
-          }
-          o = M + __log2f(Ls);
-        }
-        off[r] = o;
-      }
-      asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
-    }
-
     float m = kNegInf, l = 0.f;
-    const int row_pos = P + (my_lane % max(p.w, 1));   // stats pass: this thread's row position
+    const int row_pos = wk.P + (my_lane % max(p.w, 1));   // stats pass: this thread's row position
     const uint32_t t_lane = tmem_base + ((uint32_t)(32 * quarter) << 16) + cb * 32;
-    auto wait_full = [&](int t) {
-      const bool got = *cta_err ? true : mbar_wait(&acc_full[t % kAccBufs], (t / kAccBufs) & 1);
-      if (!__all_sync(0xffffffffu, got) && lane == 0) *cta_err = 1;
+    auto wait_full = [&](int j) {
+      const bool got = *sm.cta_err ? true : mbar_wait(&sm.acc_full[j % kAccBufs], (j / kAccBufs) & 1);
+      if (!__all_sync(0xffffffffu, got) && lane == 0) *sm.cta_err = 1;
       tc_fence_after();
     };
     // software pipeline over 16-column halves: the TMEM load of the next half
     // is in flight while the current one is reduced
     uint32_t ra[16], rb[16];
-    if (n_tiles > 0) {
+    if (n > 0) {
       wait_full(0);
       tmem_ld16(t_lane, ra);
       tmem_wait_ld16(ra);
     }
-    for (int t = 0; t < n_tiles; ++t) {
-      const int buf = t % kAccBufs;
-      const int key0 = key_begin + t * kBN;
+    for (int j = 0; j < n; ++j) {
+      const int buf = j % kAccBufs;
+      const int key0 = wk.key_begin + tile_of(j) * kBN;
       tmem_ld16(t_lane + buf * 128 + 16, rb);
       float sum = 0.f;
-      if (!kScorePass) epi_stats16(ra, key0 + cb * 32, key_end, P, row_pos, p.c, m, l);
-      else sum = epi_score16(ra, off, cb * 32, key0 + my_lane, P, p);
+      if (!kScorePass) epi_stats16(ra, key0 + cb * 32, wk.key_end, wk.P, row_pos, p.c, m, l);
+      else sum = epi_score16(ra, sm.off, cb * 32, key0 + my_lane, wk.P, p);
       tmem_wait_ld16(rb);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);    // this warp's columns of tile t are read
-      if (t + 1 < n_tiles) {
-        wait_full(t + 1);
-        tmem_ld16(t_lane + ((t + 1) % kAccBufs) * 128, ra);
+      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);   // this warp's columns of the tile are read
+      if (j + 1 < n) {
+        wait_full(j + 1);
+        tmem_ld16(t_lane + ((j + 1) % kAccBufs) * 128, ra);
       }
-      if (!kScorePass) epi_stats16(rb, key0 + cb * 32 + 16, key_end, P, row_pos, p.c, m, l);
-      else sum += epi_score16(rb, off, cb * 32 + 16, key0 + my_lane, P, p);
+      if (!kScorePass) epi_stats16(rb, key0 + cb * 32 + 16, wk.key_end, wk.P, row_pos, p.c, m, l);
+      else sum += epi_score16(rb, sm.off, cb * 32 + 16, key0 + my_lane, wk.P, p);
       if (kScorePass) {
-        const int slot = t % kXch;
-        float *xs = xch + (size_t)slot * (kColBlocks - 1) * kBN;
+        const int slot = j % kXch;
+        float *xs = sm.xch + (size_t)slot * (kColBlocks - 1) * kBN;
         const int key = key0 + my_lane;
         if (cb > 0) {
           xs[(cb - 1) * kBN + my_lane] = sum;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&xch_full[slot]);
+          if (lane == 0) mbar_arrive(&sm.xch_full[slot]);
         } else {
-          const bool ok = *cta_err ? true : mbar_wait(&xch_full[slot], (t / kXch) & 1);
-          if (!__all_sync(0xffffffffu, ok) && lane == 0) *cta_err = 1;
+          const bool ok = *sm.cta_err ? true : mbar_wait(&sm.xch_full[slot], (j / kXch) & 1);
+          if (!__all_sync(0xffffffffu, ok) && lane == 0) *sm.cta_err = 1;
           float tot = sum;
 #pragma unroll
-          for (int j = 0; j < kColBlocks - 1; ++j) tot += xs[j * kBN + my_lane];
-          if (key < key_end) p.raw[(size_t)h * p.T_total + t0 + key] = tot;
+          for (int q = 0; q < kColBlocks - 1; ++q) tot += xs[q * kBN + my_lane];
+          if (key < wk.key_end) p.raw[(size_t)wk.h * p.T_total + wk.t0 + key] = tot;
         }
       }
-      if (t + 1 < n_tiles) tmem_wait_ld16(ra);
+      if (j + 1 < n) tmem_wait_ld16(ra);
     }
     if (!kScorePass) {
       // merge the column blocks of every row, then publish the partial
-      float *xm = xch, *xl = xch + (kColBlocks - 1) * kRows;
+      float *xm = sm.xch, *xl = sm.xch + (kColBlocks - 1) * kRows;
       if (cb > 0) { xm[(cb - 1) * kRows + my_lane] = m; xl[(cb - 1) * kRows + my_lane] = l; }
       asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
       if (cb == 0 && my_lane < p.R) {
         float mn = m;
 #pragma unroll
-        for (int j = 0; j < kColBlocks - 1; ++j) mn = fmaxf(mn, xm[j * kRows + my_lane]);
+        for (int q = 0; q < kColBlocks - 1; ++q) mn = fmaxf(mn, xm[q * kRows + my_lane]);
         float ls = 0.f;
         if (mn != kNegInf) {
           ls = l * fast_exp2(m - mn);
 #pragma unroll
-          for (int j = 0; j < kColBlocks - 1; ++j) ls += xl[j * kRows + my_lane] * fast_exp2(xm[j * kRows + my_lane] - mn);
+          for (int q = 0; q < kColBlocks - 1; ++q) ls += xl[q * kRows + my_lane] * fast_exp2(xm[q * kRows + my_lane] - mn);
         }
-        p.part[((size_t)(b * p.n_kv + h) * p.n_chunks + c) * kRows + my_lane] = make_float2(mn, ls);
+        p.part[((size_t)(wk.b * p.n_kv + wk.h) * p.n_chunks + wk.c) * kRows + my_lane] = make_float2(mn, ls);
       }
     }
   }
+}
 
+// (M, L) <- merge of two running (max, sum of 2^(x - max)) pairs
+KVC_DEVINL void merge_ml(float &M, float &L, float m, float l) {
+  const float mn = fmaxf(M, m);
+  if (mn == kNegInf) return;
+  L = L * fast_exp2(M - mn) + l * fast_exp2(m - mn);
+  M = mn;
+}
+
+// Epilogue threads: off_r = M + log2(L) of every row from the stats partials
+// of all key chunks of the head (read through L2: other CTAs wrote them).
+// Four threads per row fold every fourth chunk with independent loads in
+// flight, then combine by shuffle, so the merge costs about one L2 round trip.
+KVC_DEVINL void merge_offsets(const TcParams &p, const TcSmem &sm, const TcWork &wk) {
+  static_assert(kEpiWarps * 32 == 4 * kRows, "four epilogue threads per row");
+  const int et = threadIdx.x - kEpiWarp0 * 32;
+  const int r = et >> 2, q = et & 3;
+  const float2 *pp = p.part + (size_t)(wk.b * p.n_kv + wk.h) * p.n_chunks * kRows + r;
+  const int nc = (wk.len + p.keys_per_chunk - 1) / p.keys_per_chunk;
+  float M = kNegInf, Ls = 0.f;
+  if (r < p.R) {
+    for (int cc = q; cc < nc; cc += 16) {
+      float2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = cc + 4 * u < nc ? __ldcg(pp + (size_t)(cc + 4 * u) * kRows) : make_float2(kNegInf, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) merge_ml(M, Ls, v[u].x, v[u].y);
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, M, o), l2 = __shfl_xor_sync(0xffffffffu, Ls, o);
+    merge_ml(M, Ls, m2, l2);
+  }
+  if (q == 0) sm.off[r] = (r < p.R) ? M + __log2f(Ls) : kPosInf;
+  asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
+}
+
+KVC_DEVINL bool setup_work(const TcParams &p, TcWork &wk) {
+  wk.h = blockIdx.x; wk.c = blockIdx.y; wk.b = blockIdx.z;
+  wk.t0 = p.cu_seqlens[wk.b];
+  wk.len = p.cu_seqlens[wk.b + 1] - wk.t0;
+  wk.key_begin = wk.c * p.keys_per_chunk;
+  if (wk.key_begin >= wk.len) return false;
+  wk.key_end = min(wk.len, wk.key_begin + p.keys_per_chunk);
+  wk.n_tiles = (wk.key_end - wk.key_begin + kBN - 1) / kBN;
+  wk.P = wk.len - p.w;
+  return true;
+}
+
+// Barriers, tensor memory and the window block (loaders stage it with
+// cp.async; the MMA thread waits for it before its first MMA).
+template <int D>
+KVC_DEVINL uint32_t cta_setup(const TcParams &p, const TcSmem &sm, const TcWork &wk) {
+  const int warp = warp_id();
+  if (threadIdx.x == 0) {
+    init_pass_barriers(sm, false);
+    mbar_init(sm.q_full, kLoadWarps * 32);
+    *sm.cta_err = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) { tmem_alloc(sm.tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) { tc_fence_after(); tmem_dealloc(tmem_base, 512); }
-  if (threadIdx.x == 0 && *cta_err) atomicCAS(p.err, 0, 1);
+  tc_fence_after();
+  if (warp < kLoadWarps) {
+    stage_q_async<D>(sm.sq, p, wk.b, wk.h, threadIdx.x, kLoadWarps * 32);
+    cp_async_arrive_noinc(sm.q_full);
+  } else if (warp == kMmaWarp && lane_id() == 0) {
+    if (!mbar_wait(sm.q_full, 0)) *sm.cta_err = 1;
+  }
+  return *sm.tmem_slot;
+}
+
+KVC_DEVINL void cta_teardown(const TcParams &p, const TcSmem &sm, uint32_t tmem_base) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp_id() == kMmaWarp) { tc_fence_after(); tmem_dealloc(tmem_base, 512); }
+  if (threadIdx.x == 0 && *sm.cta_err) atomicCAS(p.err, 0, 1);
+}
+
+// One pass per launch (the grid does not fit on the GPU at once).
+template <int D, bool kScorePass>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+score_tc_kernel(TcParams p) {
+  TcWork wk;
+  if (!setup_work(p, wk)) return;
+  extern __shared__ uint8_t smem_raw[];
+  const TcSmem sm = carve_smem<D>(smem_raw);
+  const uint32_t tmem_base = cta_setup<D>(p, sm, wk);
+  if (kScorePass && warp_id() >= kEpiWarp0) merge_offsets(p, sm, wk);
+  tc_pass<D, kScorePass>(p, sm, wk, tmem_base, false);
+  cta_teardown(p, sm, tmem_base);
+}
+
+// Both passes and the pool in one cooperative launch.
+template <int D>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+score_fused_kernel(TcParams p) {
+  TcWork wk;
+  if (!setup_work(p, wk)) return;
+  extern __shared__ uint8_t smem_raw[];
+  const TcSmem sm = carve_smem<D>(smem_raw);
+  const uint32_t tmem_base = cta_setup<D>(p, sm, wk);
+  const int nc = (wk.len + p.keys_per_chunk - 1) / p.keys_per_chunk;
+  int *ctr = p.sync + (size_t)(wk.b * p.n_kv + wk.h) * 4;
+
+  tc_pass<D, false>(p, sm, wk, tmem_base, false);
+
+  // every chunk of this head has published its stats partial
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!arrive_and_wait(&ctr[0], nc)) *sm.cta_err = 1;
+    init_pass_barriers(sm, true);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp_id() >= kEpiWarp0) merge_offsets(p, sm, wk);
+
+  tc_pass<D, true>(p, sm, wk, tmem_base, true);
+
+  // every chunk of this head has written its raw scores: pool the chunk
+  __syncthreads();
+  if (threadIdx.x == 0 && !arrive_and_wait(&ctr[1], nc)) *sm.cta_err = 1;
+  __syncthreads();
+  {
+    const float *src = p.raw + (size_t)wk.h * p.T_total + wk.t0;
+    float *dst = p.scores + (size_t)wk.h * p.T_total + wk.t0;
+    const int r = p.pool_r;
+    for (int j = wk.key_begin + threadIdx.x; j < wk.key_end; j += kThreadsTC) {
+      float v = kPosInf;
+      if (j < wk.P) {
+        const int lo = max(0, j - r), hi = min(wk.P - 1, j + r);
+        v = __ldcg(src + lo);
+        for (int q = lo + 1; q <= hi; ++q) v = fmaxf(v, __ldcg(src + q));
+      }
+      dst[j] = v;
+    }
+  }
+
+  // the last CTA of this head to leave resets the counters for the next call
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(&ctr[2], 1) == nc - 1) { ctr[0] = 0; ctr[1] = 0; ctr[2] = 0; }
+  cta_teardown(p, sm, tmem_base);
 }
 
 template <int D>
@@ -386,17 +562,32 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
   p.cu_seqlens = a.cu_seqlens;
   p.part = a.part;
   p.raw = a.raw;
+  p.scores = a.scores;
+  p.sync = a.sync;
   p.err = a.err;
   p.n_h = a.n_h; p.n_kv = a.n_kv; p.G = a.n_h / a.n_kv; p.w = a.w; p.R = p.G * a.w;
   p.n_chunks = a.n_chunks; p.keys_per_chunk = a.keys_per_chunk; p.T_total = a.T_total;
+  p.pool_r = a.pool_k / 2;
   p.c = a.scale * kLog2e;
   const int smem = TcLayout<D>::kAlloc;
-  cudaError_t e;
-  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, false>, smem)))
-    return e;
-  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, true>, smem)))
-    return e;
   dim3 grid(a.n_kv, a.n_chunks, a.n_seqs);
+  cudaError_t e;
+  if (a.fused) {
+    if ((e = ensure_smem_limit((const void *)score_fused_kernel<D>, smem))) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreadsTC);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, score_fused_kernel<D>, p);
+  }
+  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, false>, smem))) return e;
+  if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, true>, smem))) return e;
   score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(p);
   if ((e = cudaGetLastError())) return e;
   score_tc_kernel<D, true><<<grid, kThreadsTC, smem, st>>>(p);

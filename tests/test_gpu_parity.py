@@ -36,6 +36,19 @@ def test_bf16_tensor_core_ragged(lengths):
     run_and_check_compress("bf16", lengths, 32, 8, 128, 32, 7, 200, seed=1234)
 
 
+def test_bf16_tensor_core_split_launches():
+    """20 sequences x 8 KV heads = 160 work items: more than fit on the GPU at
+    once, so the two passes and the pool run as separate launches."""
+    lengths = synth.ragged_lengths(4242, 20, 40, 700).tolist()
+    run_and_check_compress("bf16", lengths, 32, 8, 128, 32, 7, 96, seed=4243)
+
+
+def test_bf16_fused_repeated_calls():
+    """The single cooperative launch, three times on the same workspace: its
+    arrival counters must come back to zero after every call."""
+    run_and_check_compress("bf16", [3000, 1500], 32, 8, 128, 32, 7, 300, seed=4244, repeat=3)
+
+
 def test_bf16_tensor_core_small_block_d64():
     """G*w = 16 rows padded to the 128-row tile; d_h 64 (one swizzle atom)."""
     run_and_check_compress("bf16", [513, 64, 200], 8, 4, 64, 8, 3, 40, seed=77)
