@@ -129,14 +129,18 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
     const int r1 = (int)(min(x_end, u0 + len) - u0);
     const int u = b * p.n_kv + h;
 
-    // query slices of the G heads of h: element d = j * (LPR * EPC) + sl * EPC + i of chunk j
+    // query slices of the G heads of h: element d = j * (LPR * EPC) + sl * EPC + i of chunk j.
+    // Slot g holds head g ^ xq: with this lane-dependent order every stage of
+    // the reduce-scatter below keeps the low half of the slots and sends the
+    // high half, so it needs no selects.
+    const int xq = (G <= LPR) ? (sl / (LPR / G)) & (G - 1) : 0;
     float qr[G][16];
     const T *qb = static_cast<const T *>(p.q) + ((size_t)b * p.n_h + (size_t)h * G) * D;
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
       for (int j = 0; j < NCH; ++j) {
-        unpack16<T>(ld_nc16(qb + (size_t)g * D + j * (LPR * EPC) + sl * EPC), &qr[g][j * EPC]);
+        unpack16<T>(ld_nc16(qb + (size_t)(g ^ xq) * D + j * (LPR * EPC) + sl * EPC), &qr[g][j * EPC]);
 #pragma unroll
         for (int i = 0; i < EPC; ++i) qr[g][j * EPC + i] *= p.c;
       }
@@ -157,56 +161,55 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
     const size_t step_stride = (size_t)RPW * rstride;
     const T *k_any = kb + (size_t)r0 * rstride, *v_any = vb + (size_t)r0 * rstride;   // a valid dummy source
     const T *kq = kb + (size_t)(r0 + rg) * rstride, *vq = vb + (size_t)(r0 + rg) * rstride;
+    // ring pointers: the slot of the next prefetched step and of the next consumed one
+    uint8_t *const ring_end = ring + kRing * RG::kStepBytes;
+    uint8_t *pf_dst = ring;
+    const uint8_t *src = ring;
+    int pf_row = r0 + rg;        // this lane's row of the next prefetched step
+    auto prefetch = [&]() {
+      // zero-filled (no read) past the segment; one cp.async group per step
+      const bool ok = pf_row < r1;
+      const T *ks = ok ? kq : k_any, *vs = ok ? vq : v_any;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        cp_async16(pf_dst + j * 512, ks + j * (LPR * EPC), ok);
+        cp_async16(pf_dst + (NCH + j) * 512, vs + j * (LPR * EPC), ok);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      kq += step_stride;
+      vq += step_stride;
+      pf_row += RPW;
+      pf_dst += RG::kStepBytes;
+      if (pf_dst == ring_end) pf_dst = ring;
+    };
+#pragma unroll 1
+    for (int s = 0; s < kRing - 1; ++s) prefetch();
     int row = r0 + rg;
 #pragma unroll 1
-    for (int s = 0; s < kRing - 1 + n_steps; ++s) {
-      {
-        // prefetch step s (zero-filled past the segment); one cp.async group per step
-        const bool valid = s < n_steps && row < r1;
-        const T *ks = valid ? kq : k_any, *vs = valid ? vq : v_any;
-        uint8_t *dst = ring + ((unsigned)s & (kRing - 1)) * RG::kStepBytes;
-#pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-          cp_async16(dst + j * 512, ks + j * (LPR * EPC), valid);
-          cp_async16(dst + (NCH + j) * 512, vs + j * (LPR * EPC), valid);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        kq += step_stride;
-        vq += step_stride;
-        row += RPW;
-      }
-      const int st = s - (kRing - 1);           // step consumed in this iteration
-      if (st < 0) continue;
+    for (int st = 0; st < n_steps; ++st) {
+      prefetch();                               // step st + kRing - 1
       asm volatile("cp.async.wait_group %0;" :: "n"(kRing - 1) : "memory");
-      const uint8_t *src = ring + ((unsigned)st & (kRing - 1)) * RG::kStepBytes;
-      const bool valid = r0 + st * RPW + rg < r1;
+      const bool valid = row < r1;
+      row += RPW;
       float kf[16];
 #pragma unroll
       for (int j = 0; j < NCH; ++j) unpack16<T>(*reinterpret_cast<const uint4 *>(src + j * 512), &kf[j * EPC]);
       float sc[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          ffma2(a0, a1, qr[g][e], qr[g][e + 1], kf[e], kf[e + 1]);
-          ffma2(a2, a3, qr[g][e + 2], qr[g][e + 3], kf[e + 2], kf[e + 3]);
-        }
-        sc[g] = (a0 + a1) + (a2 + a3);
+        for (int e = 0; e < 16; e += 2) ffma2(a0, a1, qr[g][e], qr[g][e + 1], kf[e], kf[e + 1]);
+        sc[g] = a0 + a1;
       }
       if constexpr (G <= LPR) {
         // reduce-scatter over the LPR lanes of the row: afterwards this lane
-        // holds the full logit of one head, hs = sl / (LPR / G)
+        // holds the full logit of one head, xq = sl / (LPR / G); slot j holds
+        // head j ^ xq, so the partner across bit o needs exactly our high half
 #pragma unroll
-        for (int k = G, o = LPR / 2; k > 1; k >>= 1, o >>= 1) {
-          const bool up = (sl & o) != 0;
+        for (int k = G, o = LPR / 2; k > 1; k >>= 1, o >>= 1)
 #pragma unroll
-          for (int j = 0; j < k / 2; ++j) {
-            const float mine = up ? sc[k / 2 + j] : sc[j];
-            const float other = up ? sc[j] : sc[k / 2 + j];
-            sc[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
-          }
-        }
+          for (int j = 0; j < k / 2; ++j) sc[j] += __shfl_xor_sync(0xffffffffu, sc[k / 2 + j], o);
 #pragma unroll
         for (int o = (LPR / G) / 2; o >= 1; o >>= 1) sc[0] += __shfl_xor_sync(0xffffffffu, sc[0], o);
         const float s_my = sc[0];
@@ -274,6 +277,8 @@ __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p
           }
         }
       }
+      src += RG::kStepBytes;
+      if (src == ring_end) src = ring;
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 
