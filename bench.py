@@ -168,9 +168,12 @@ def run_ours(args):
         torch.sum(sweep, dim=0, out=sink)
 
     stream = torch.cuda.current_stream(dev)
+    from kv_cache_compression_score_b200 import kvc
 
-    # the four C-ABI calls of a step, each captured once in a CUDA graph so the
-    # timed region measures device time, not Python/ctypes enqueue time
+    # the C-ABI calls of a step: score -> select -> gather captured as one CUDA
+    # graph (the headline), decode as a second; each call also gets a graph of
+    # its own for the per-call breakdown.  Graphs keep Python/ctypes enqueue
+    # time out of the timed region.
     calls = [lambda: comp.score(q_win, k), lambda: comp.select(), lambda: comp.gather(k, v),
              lambda: dec.run(qd, kc_all, vc_all, off, ln)]
     side = torch.cuda.Stream(dev)
@@ -180,48 +183,78 @@ def run_ours(args):
             fn()
     stream.wait_stream(side)
     torch.cuda.synchronize()
-    graphs = []
-    for fn in calls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        graphs.append(g)
-    torch.cuda.synchronize()
 
-    def step(evs=None):
-        if evs: evs[0].record(stream)
-        for j, g in enumerate(graphs):
-            g.replay()
-            if evs: evs[j + 1].record(stream)
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        n0 = kvc.kvc_launch_count()
+        with torch.cuda.graph(g):
+            for fn in fns:
+                fn()
+        return g, kvc.kvc_launch_count() - n0
+
+    g_ssg, n_ssg = capture(calls[:3])
+    g_dec, n_dec = capture(calls[3:])
+    per_call = [capture([fn])[0] for fn in calls]
+    torch.cuda.synchronize()
+    kernels_per_step = n_ssg + n_dec
 
     for _ in range(args.warmup):
         flush_l2()
-        step()
+        g_ssg.replay()
+        g_dec.replay()
     torch.cuda.synchronize()
     assert comp.device_error_word() == 0, "device error word set"
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
     for i in range(args.steps):
         flush_l2()
-        step(evs[i])
+        evs[i][0].record(stream)
+        g_ssg.replay()
+        evs[i][1].record(stream)
+        g_dec.replay()
+        evs[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     t_wall = time.perf_counter() - t_wall
     clocks = sampler.stop()
+    assert comp.device_error_word() == 0, "device error word set"
 
-    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])  # ms
+    ssg_samples = [evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps)]   # ms
+    t_ssg = float(np.mean(ssg_samples))
+    t_dec = float(np.mean([evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)]))
+    t_step = t_ssg + t_dec
+
+    # the same three calls without graph capture (direct C-ABI calls, device-resident inputs)
+    uevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2()
+        uevs[i][0].record(stream)
+        for fn in calls[:3]:
+            fn()
+        uevs[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_ssg_direct = float(np.mean([a.elapsed_time(b) for a, b in uevs]))
+
+    # per-call breakdown (same flush between steps; separate graphs per call)
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2()
+        bevs[i][0].record(stream)
+        for j, g in enumerate(per_call):
+            g.replay()
+            bevs[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    per = np.array([[bevs[i][j].elapsed_time(bevs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
     mean = per.mean(axis=0)
-    t_ssg = float(mean[:3].sum())
-    t_step = float(mean.sum())
-    t_dec = float(mean[3])
     t_ssg, t_step, t_dec = max_over_ranks([t_ssg, t_step, t_dec], dev)
+    mean = np.array(max_over_ranks(list(mean), dev))
 
     # ---- e2e: the same path through the C ABI with pinned host buffers
     e2e = run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush_l2)
@@ -253,19 +286,24 @@ def run_ours(args):
             "config": {"workload": cfg["name"], "n_h": n_h, "n_kv": n_kv, "d_h": d, "seq_len": S, "window": w,
                        "pool": cfg["pool_k"], "budget": B, "decode_batch": nb,
                        "l2": "flushed between steps (256 MiB write + 256 MiB read sweep, outside the timed events)",
-                       "launch": "one CUDA graph per C-ABI call, replayed back to back",
+                       "launch": "score+select+gather as one CUDA graph (timed for value), decode as a second; "
+                                 "breakdown_us from one graph per call",
                        "parallelism": f"replicas x{world}"},
             "gbs": round(ssg_gbs, 1),
             "decode": {"gbs": round(dec_gbs, 1), "us": round(t_dec * 1e3, 2), "frac_of_8000": round(dec_gbs / 8000, 3)},
             "breakdown_us": {c: round(float(calls[c][0]) * 1e3, 2) for c in calls},
             "ssg_us": round(t_ssg * 1e3, 2),
+            "ssg_us_stats": {"graph_median": round(float(np.median(ssg_samples)) * 1e3, 2),
+                             "graph_min": round(float(np.min(ssg_samples)) * 1e3, 2),
+                             "uncaptured_mean": round(t_ssg_direct * 1e3, 2)},
             "ssg_frac_of_8000": round(ssg_gbs / 8000, 3),
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / hbm, 3),
                          "traffic": traffic},
             "e2e": {"value": round(world * S / (e2e["t_ms"] * 1e-3) / 1e3, 2), "unit": "K-tok/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": kernels_per_step * args.steps,
+            "kernels_per_step": kernels_per_step,
             "clocks": clocks,
             "wall_s_timed_region": round(t_wall, 3),
         }
@@ -312,16 +350,22 @@ def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, 
     return {"t_ms": t, "h2d": h2d, "d2h": d2h}
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch of the dominant call from the committed ncu summary, if current."""
+def load_traffic(call):
+    """DRAM bytes per launch of a call's kernel from the committed ncu summary
+    (profiles/traffic.json), or None once the kernel's source has changed
+    since the counters were taken (its sha256 no longer matches)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        e = d.get(kernel)
-        if e and e.get("current", False):
-            return e.get("bytes_per_launch")
-    return None
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        e = json.load(f).get(call)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != e["sha256"]:
+        return None
+    return e["bytes_per_launch"]
 
 
 # ----------------------------------------------------------- oracle arm

@@ -67,7 +67,8 @@ typedef enum kvc_status {
   KVC_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or count */
   KVC_ERR_UNSUPPORTED = 2,  /* valid request outside the kernels' shapes/dtypes */
   KVC_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
-  KVC_ERR_CUDA = 4          /* a CUDA runtime call or launch failed */
+  KVC_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  KVC_ERR_DEVICE_CHECK = 5  /* a workspace's device error word is set (kvc_check_workspace) */
 } kvc_status;
 
 typedef enum kvc_dtype {
@@ -77,6 +78,20 @@ typedef enum kvc_dtype {
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int kvc_version(void);
+
+/* Number of kernels this library has enqueued in this process (kernels
+ * recorded into a CUDA graph under stream capture count once, at capture).
+ * For launch accounting by callers; the pages have no counterpart. */
+int64_t kvc_launch_count(void);
+
+/* Read a workspace's device error word (its first int32).  The one
+ * synchronous call of the library: it waits for `stream`, then copies the
+ * word to the host; it allocates nothing.  Returns KVC_OK when the word is
+ * zero, KVC_ERR_DEVICE_CHECK when a kernel that used this workspace gave up
+ * a bounded wait (the results of the calls since the workspace was last
+ * zeroed are invalid; zero it again before reuse), KVC_ERR_INVALID_ARG for a
+ * NULL or misaligned ws, KVC_ERR_CUDA when the copy or the wait failed. */
+kvc_status kvc_check_workspace(const void *ws, kvc_stream_t stream);
 
 /* Static text for a status code. */
 const char *kvc_status_string(int status);

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -144,6 +145,9 @@ kvc_status plan_decode(kvc_dtype dt, int batch, int n_h, int n_kv, int d_h, int 
 }  // namespace
 
 namespace kvc {
+std::atomic<int64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 cudaError_t ensure_smem_limit(const void *fn, int bytes) {
   static std::mutex mu;
   static std::vector<std::pair<std::pair<const void *, int>, int>> done;   // ((fn, device), bytes)
@@ -163,6 +167,20 @@ extern "C" {
 
 int kvc_version(void) { return 100; }
 
+int64_t kvc_launch_count(void) { return kvc::g_launches.load(std::memory_order_relaxed); }
+
+kvc_status kvc_check_workspace(const void *ws, kvc_stream_t stream) {
+  if (!aligned16(ws)) return fail(KVC_ERR_INVALID_ARG, "ws must be non-NULL and 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "waiting for the stream");
+  if (word != 0) return fail(KVC_ERR_DEVICE_CHECK, "device error word is %d: a bounded wait gave up", word);
+  return KVC_OK;
+}
+
 const char *kvc_status_string(int status) {
   switch (status) {
     case KVC_OK: return "KVC_OK";
@@ -170,6 +188,7 @@ const char *kvc_status_string(int status) {
     case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
     case KVC_ERR_WORKSPACE: return "KVC_ERR_WORKSPACE";
     case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+    case KVC_ERR_DEVICE_CHECK: return "KVC_ERR_DEVICE_CHECK";
     default: return "KVC_ERR_UNKNOWN";
   }
 }

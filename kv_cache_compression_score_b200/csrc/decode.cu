@@ -83,6 +83,7 @@ KVC_DEVINL int64_t owner(int64_t x, int64_t R, int64_t NW) {
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreadsDec, 1) gqa_decode_streamk(DecParams p) {
+  grid_dependency_wait();
   using RG = DecRing<T>;
   constexpr int LPR = D / 16;              // lanes per row
   constexpr int RPW = 32 / LPR;            // rows per warp step
@@ -411,8 +412,8 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t st) {
   p.q = a.q; p.kc = a.k_c; p.vc = a.v_c; p.row_off = a.row_off; p.kv_len = a.kv_len; p.out = a.out;
   p.part = a.part; p.tickets = a.tickets; p.batch = a.batch; p.n_h = a.n_h; p.n_kv = a.n_kv;
   p.slots = a.n_chunks; p.c = a.scale * kLog2e;
-  gqa_decode_streamk<T, D, G><<<kNumSMs, kThreadsDec, smem, st>>>(p);
-  return cudaGetLastError();
+  count_launch();
+  return launch_pdl(gqa_decode_streamk<T, D, G>, dim3(kNumSMs), dim3(kThreadsDec), (size_t)smem, st, p);
 }
 
 template <typename T, int D>

@@ -19,6 +19,8 @@ __global__ void __launch_bounds__(kGatherThreads)
 gather_kv_kernel(const uint8_t *__restrict__ k, const uint8_t *__restrict__ v, uint8_t *__restrict__ k_out,
                  uint8_t *__restrict__ v_out, const int32_t *__restrict__ idx, const int *__restrict__ cu_seqlens,
                  const int *__restrict__ cu_budget, int n_kv, int vec_per_head, int total_budget) {
+  grid_dependency_wait();
+  allow_dependents();
   const int b = blockIdx.y;
   const int t0 = cu_seqlens[b], len = cu_seqlens[b + 1] - t0;
   const int cb = cu_budget[b], kept = cu_budget[b + 1] - cb;
@@ -63,6 +65,8 @@ gather_kv_kernel(const uint8_t *__restrict__ k, const uint8_t *__restrict__ v, u
 __global__ void __launch_bounds__(kGatherThreads)
 gather_hidden_kernel(const uint8_t *__restrict__ hidden, uint8_t *__restrict__ out, const int32_t *__restrict__ idx,
                      int n_rows, int vec_per_row, int n_src) {
+  grid_dependency_wait();
+  allow_dependents();
   const long long n_items = (long long)n_rows * vec_per_row;
   for (long long base = (long long)blockIdx.x * kGatherThreads * kGatherUnroll + threadIdx.x; base < n_items;
        base += (long long)gridDim.x * kGatherThreads * kGatherUnroll) {
@@ -99,10 +103,10 @@ cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_ou
   if (blocks < 1) blocks = 1;
   if (blocks > 65535) blocks = 65535;
   dim3 grid((unsigned)blocks, n_seqs);
-  gather_kv_kernel<<<grid, kGatherThreads, 0, st>>>(
-      static_cast<const uint8_t *>(k), static_cast<const uint8_t *>(v), static_cast<uint8_t *>(k_out),
-      static_cast<uint8_t *>(v_out), idx, cu_seqlens, cu_budget, n_kv, vph, total_budget);
-  return cudaGetLastError();
+  count_launch();
+  return launch_pdl(gather_kv_kernel, grid, dim3(kGatherThreads), 0, st, static_cast<const uint8_t *>(k),
+                    static_cast<const uint8_t *>(v), static_cast<uint8_t *>(k_out), static_cast<uint8_t *>(v_out), idx,
+                    cu_seqlens, cu_budget, n_kv, vph, total_budget);
 }
 
 cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int n_rows, int row_bytes, int n_src,
@@ -112,9 +116,9 @@ cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int
   const long long items = (long long)n_rows * vpr;
   long long blocks = (items + kGatherThreads * kGatherUnroll - 1) / (kGatherThreads * kGatherUnroll);
   if (blocks > 65535) blocks = 65535;
-  gather_hidden_kernel<<<(unsigned)blocks, kGatherThreads, 0, st>>>(
-      static_cast<const uint8_t *>(hidden), static_cast<uint8_t *>(out), idx, n_rows, vpr, n_src);
-  return cudaGetLastError();
+  count_launch();
+  return launch_pdl(gather_hidden_kernel, dim3((unsigned)blocks), dim3(kGatherThreads), 0, st,
+                    static_cast<const uint8_t *>(hidden), static_cast<uint8_t *>(out), idx, n_rows, vpr, n_src);
 }
 
 }  // namespace kvc

@@ -65,6 +65,17 @@ KVC_DEVINL uint32_t smem_u32(const void *p) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream is still
+// running; grid_dependency_wait() blocks until that kernel has completed and
+// its memory is visible (a no-op without such a predecessor), so a dependent
+// kernel calls it before its first global access.  allow_dependents() lets
+// the next kernel of the stream begin launching early.
+// ---------------------------------------------------------------------------
+KVC_DEVINL void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+KVC_DEVINL void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// ---------------------------------------------------------------------------
 // mbarrier (shared-memory transaction barrier) with bounded waits.  A wait
 // that runs past its time limit returns false; the caller records an error
 // code, stops issuing work and leaves through its normal exit path.

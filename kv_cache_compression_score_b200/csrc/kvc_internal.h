@@ -74,6 +74,27 @@ int decode_slots(int max_kv_len);
 }  // namespace kvc
 
 namespace kvc {
+// Host-side count of kernels this library enqueued (or recorded into a graph
+// under stream capture); every launch site calls it once per launch.
+void count_launch();
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel of the stream finishes; it calls grid_dependency_wait()
+// before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
 // Raise a kernel's dynamic shared-memory limit once per device (a host call
 // kept out of the per-launch path, so launches can be captured in graphs).
 cudaError_t ensure_smem_limit(const void *fn, int bytes);

@@ -530,6 +530,8 @@ KVC_DEVINL void cluster_topk_ascending(const float *__restrict__ src, int n, int
 __global__ void __launch_bounds__(kCThreads)
 select_topk_cluster(const float *__restrict__ scores, int32_t *__restrict__ idx, const int *__restrict__ cu_seqlens,
                     const int *__restrict__ cu_budget, int T_total, int total_budget, int w, int budget) {
+  grid_dependency_wait();
+  allow_dependents();
   const int h = blockIdx.x / kClu, b = blockIdx.y;
   const uint32_t rank = cluster_rank();
   const int t0 = cu_seqlens[b], len = cu_seqlens[b + 1] - t0;
@@ -548,6 +550,8 @@ select_topk_cluster(const float *__restrict__ scores, int32_t *__restrict__ idx,
 
 __global__ void __launch_bounds__(kCThreads)
 tsp_select_cluster(const float *__restrict__ pooled, int S, int w, int k_tsp, int32_t *__restrict__ idx_out) {
+  grid_dependency_wait();
+  allow_dependents();
   const uint32_t rank = cluster_rank();
   const int P = S - w;
   extern __shared__ uint32_t csel_cache[];
@@ -567,6 +571,7 @@ cudaError_t pool_prefix(const float *raw, float *scores, const int32_t *cu_seqle
                         int T_total, int max_len, int w, int pool_k, cudaStream_t st) {
   dim3 grid((max_len + kPoolTile - 1) / kPoolTile, n_kv, n_seqs);
   pool_prefix_kernel<<<grid, kPoolThreads, 0, st>>>(raw, scores, cu_seqlens, T_total, w, (pool_k - 1) / 2);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -575,6 +580,7 @@ cudaError_t tsp_pool(const float *raw, int n_rows, int S, int w, int pool_k, flo
   if (P <= 0) return cudaSuccess;
   tsp_pool_kernel<<<(P + kPoolTile - 1) / kPoolTile, kPoolThreads, 0, st>>>(raw, n_rows, S, w, (pool_k - 1) / 2,
                                                                             pooled);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -586,13 +592,16 @@ static cudaError_t launch_cluster(const void *fn, dim3 grid, size_t smem, cudaSt
   cfg.blockDim = dim3(kCThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kClu;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
+  count_launch();
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 

@@ -263,9 +263,11 @@ static cudaError_t launch_simt(const ScoreArgs &a, cudaStream_t st) {
   dim3 grid(a.n_chunks, a.n_kv, a.n_seqs);
   score_stats_simt<T, D><<<grid, kThreads, smem, st>>>(
       static_cast<const T *>(a.q_win), static_cast<const T *>(a.k), a.cu_seqlens, s, a.part);
+  count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   score_raw_simt<T, D><<<grid, kThreads, smem, st>>>(
       static_cast<const T *>(a.q_win), static_cast<const T *>(a.k), a.cu_seqlens, s, a.part, a.raw, a.T_total);
+  count_launch();
   return cudaGetLastError();
 }
 

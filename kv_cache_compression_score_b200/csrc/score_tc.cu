@@ -505,6 +505,7 @@ score_tc_kernel(TcParams p) {
 template <int D>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 score_fused_kernel(TcParams p) {
+  allow_dependents();
   TcWork wk;
   if (!setup_work(p, wk)) return;
   extern __shared__ uint8_t smem_raw[];
@@ -584,13 +585,16 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    count_launch();
     return cudaLaunchKernelEx(&cfg, score_fused_kernel<D>, p);
   }
   if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, false>, smem))) return e;
   if ((e = ensure_smem_limit((const void *)score_tc_kernel<D, true>, smem))) return e;
   score_tc_kernel<D, false><<<grid, kThreadsTC, smem, st>>>(p);
+  count_launch();
   if ((e = cudaGetLastError())) return e;
   score_tc_kernel<D, true><<<grid, kThreadsTC, smem, st>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -17,12 +17,16 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvc.so")
 
 KVC_F32, KVC_BF16 = 0, 1
+# kvc_status
+KVC_OK, KVC_ERR_INVALID_ARG, KVC_ERR_UNSUPPORTED, KVC_ERR_WORKSPACE, KVC_ERR_CUDA, KVC_ERR_DEVICE_CHECK = range(6)
 
 # entry points declared in include/kvc.h, with their ctypes signatures
 _c_int, _c_i64, _c_u64, _c_sz, _c_f, _c_p = (ctypes.c_int, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t,
                                              ctypes.c_float, ctypes.c_void_p)
 SIGNATURES = {
     "kvc_version": (_c_int, []),
+    "kvc_launch_count": (_c_i64, []),
+    "kvc_check_workspace": (_c_int, [_c_p, _c_p]),
     "kvc_status_string": (ctypes.c_char_p, [_c_int]),
     "kvc_last_error": (ctypes.c_char_p, []),
     "kvc_cache_bytes": (_c_u64, [_c_int, _c_i64, _c_int, _c_int, _c_int]),
@@ -104,6 +108,20 @@ def dtype_code(t) -> int:
 # ------------------------------------------------------------------ host side
 def kvc_version() -> int:
     return lib().kvc_version()
+
+
+def kvc_launch_count() -> int:
+    """Kernels this library has enqueued in this process (graph captures count once)."""
+    return int(lib().kvc_launch_count())
+
+
+def kvc_check_workspace(ws, stream=None) -> int:
+    """Status of a workspace's device error word after waiting for the stream:
+    KVC_OK (0) or KVC_ERR_DEVICE_CHECK (5); other failures raise KvcError."""
+    st = int(lib().kvc_check_workspace(_dptr(ws), _stream(stream)))
+    if st not in (KVC_OK, KVC_ERR_DEVICE_CHECK):
+        _check(st)
+    return st
 
 
 def kvc_cache_bytes(L: int, S: int, n_kv: int, d_h: int, b: int) -> int:

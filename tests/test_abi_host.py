@@ -127,3 +127,13 @@ def test_select_gather_decode_tsp_reject_before_launch(L):
                                    None) == INVALID
     assert L.kvc_tsp_select_gather(kvc.KVC_BF16, 100, 8, 32, 7, 10, P16, P16, 4, P16, P16, P16, 1 << 20,
                                    None) == UNSUPPORTED
+
+
+def test_check_workspace_and_launch_count_need_no_gpu_to_validate(L):
+    """kvc_check_workspace rejects a NULL workspace before any CUDA call; the
+    launch counter is readable without a device."""
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_check_workspace(None, stream=0)
+    assert e.value.status == kvc.KVC_ERR_INVALID_ARG
+    assert L.kvc_status_string(kvc.KVC_ERR_DEVICE_CHECK) == b"KVC_ERR_DEVICE_CHECK"
+    assert kvc.kvc_launch_count() >= 0

@@ -49,6 +49,19 @@ def test_bf16_fused_repeated_calls():
     run_and_check_compress("bf16", [3000, 1500], 32, 8, 128, 32, 7, 300, seed=4244, repeat=3)
 
 
+def test_check_workspace_reads_the_device_error_word():
+    """kvc_check_workspace: clear after a healthy call; KVC_ERR_DEVICE_CHECK
+    once the error word is nonzero (planted from the host, no fault)."""
+    from kv_cache_compression_score_b200 import kvc
+    r = run_and_check_compress("bf16", [600], 32, 8, 128, 32, 7, 100, seed=4245)
+    ws = r["comp"].buf.ws
+    assert kvc.kvc_check_workspace(ws) == kvc.KVC_OK
+    ws[:4].view(torch.int32).fill_(1)
+    assert kvc.kvc_check_workspace(ws) == kvc.KVC_ERR_DEVICE_CHECK
+    ws[:4].view(torch.int32).fill_(0)
+    assert kvc.kvc_check_workspace(ws) == kvc.KVC_OK
+
+
 def test_bf16_tensor_core_small_block_d64():
     """G*w = 16 rows padded to the 128-row tile; d_h 64 (one swizzle atom)."""
     run_and_check_compress("bf16", [513, 64, 200], 8, 4, 64, 8, 3, 40, seed=77)
