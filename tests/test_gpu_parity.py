@@ -62,6 +62,29 @@ def test_check_workspace_reads_the_device_error_word():
     assert kvc.kvc_check_workspace(ws) == kvc.KVC_OK
 
 
+def test_fused_wait_gives_up_and_reports():
+    """A cross-CTA wait that can never complete (its arrival counter planted
+    far below zero from the host: no fault, no trap) gives up after its time
+    limit; the call returns, the device error word reads back as
+    KVC_ERR_DEVICE_CHECK, the counters are left at zero, and the context stays
+    usable: a rerun on the re-zeroed workspace matches the oracle."""
+    from kv_cache_compression_score_b200 import kvc
+    lengths = [2000]
+    bt = synth.packed_batch(4246, lengths, 32, 8, 128, 32, "bf16", 0.0, 3.0)
+    q, k, v = (to_device(bt[x], "bf16") for x in ("q_win", "k", "v"))
+    comp = Compressor("bf16", lengths, 32, 8, 128, 32, 7, 200)
+    ctr = comp.buf.ws[256:256 + 16 * 8].view(torch.int32)
+    ctr[0] = -1 << 20                                   # head 0's stats barrier can never fill
+    comp.score(q, k)
+    assert kvc.kvc_check_workspace(comp.buf.ws) == kvc.KVC_ERR_DEVICE_CHECK
+    assert int(ctr.abs().sum().item()) == 0             # the last CTA of each head reset them
+    comp.buf.ws.zero_()
+    comp.score(q, k)
+    assert kvc.kvc_check_workspace(comp.buf.ws) == kvc.KVC_OK
+    raw_o = O.raw_scores(bt["q_win"], bt["k"], bt["cu_seqlens"], 32, 8, 32, "bf16")
+    assert_scores_close(comp.buf.scores_raw.cpu().numpy(), raw_o, what="raw scores after recovery")
+
+
 def test_bf16_tensor_core_small_block_d64():
     """G*w = 16 rows padded to the 128-row tile; d_h 64 (one swizzle atom)."""
     run_and_check_compress("bf16", [513, 64, 200], 8, 4, 64, 8, 3, 40, seed=77)
