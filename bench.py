@@ -4,20 +4,21 @@
 
 One step = one pass of the whole path over one batch of seeded synthetic input
 (Llama-3-8B-shaped layer: n_h 32, n_kv 8, d_h 128, bf16, S 32768, window 32,
-pool 7, budget 2048, 1% of keys boosted):
-  kvc_score_window -> kvc_select_topk -> kvc_gather_kv for one sequence, then
-  kvc_gqa_decode_attn for a batch of 16 compact caches (cache 0 is the one the
-  step's gather writes; caches 1..15 are seeded stand-ins of the same shape).
+pool 7, budget 2048, 1% of keys boosted): kvc_compress_window (score, select
+and gather of one sequence in one call), then kvc_gqa_decode_attn for a batch
+of 16 compact caches (cache 0 is the one the step's gather writes; caches
+1..15 are seeded stand-ins of the same shape).
 
 value = K tokens/s of score + select + gather (S / time / 1e3), whole job over
-all ranks; decode GB/s and the per-call breakdown are extra keys.  Each C-ABI
-call is captured once in a CUDA graph and the graphs are replayed back to back,
-so the timed region holds device work only; the e2e leg calls the C ABI
-directly with host buffers.  Timing: CUDA
-events around every step on the launching stream, L2 flushed (256 MiB write,
-then a 256 MiB read sweep so no dirty lines are left)
-between steps outside the events, max over ranks.  With N > 1 every rank runs
-its own sequences (weak scaling, no collective on the data path).
+all ranks; decode GB/s and the per-call breakdown (including the three
+separate calls kvc_score_window, kvc_select_topk, kvc_gather_kv) are extra
+keys.  Each call is captured once in a CUDA graph and replayed, so the timed
+region holds device work only; ssg_us_stats adds an uncaptured timing, and
+the e2e leg calls the C ABI directly with host buffers.  Timing: CUDA events
+around every step on the launching stream, L2 flushed (256 MiB write, then a
+256 MiB read sweep so no dirty lines are left) between steps outside the
+events, max over ranks.  With N > 1 every rank runs its own sequences (weak
+scaling, no collective on the data path).
 
 --impl reference runs the fp64 CPU oracle on the same workload and metric
 (rank 0 only; the pages ship no code, so the oracle is the reference arm).
@@ -175,7 +176,7 @@ def run_ours(args):
     # its own for the per-call breakdown.  Graphs keep Python/ctypes enqueue
     # time out of the timed region.
     calls = [lambda: comp.score(q_win, k), lambda: comp.select(), lambda: comp.gather(k, v),
-             lambda: dec.run(qd, kc_all, vc_all, off, ln)]
+             lambda: dec.run(qd, kc_all, vc_all, off, ln), lambda: comp.compress(q_win, k, v)]
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
@@ -192,8 +193,8 @@ def run_ours(args):
                 fn()
         return g, kvc.kvc_launch_count() - n0
 
-    g_ssg, n_ssg = capture(calls[:3])
-    g_dec, n_dec = capture(calls[3:])
+    g_ssg, n_ssg = capture(calls[4:5])          # kvc_compress_window: score + select + gather in one call
+    g_dec, n_dec = capture(calls[3:4])
     per_call = [capture([fn])[0] for fn in calls]
     torch.cuda.synchronize()
     kernels_per_step = n_ssg + n_dec
@@ -231,19 +232,18 @@ def run_ours(args):
     t_dec = float(np.mean([evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)]))
     t_step = t_ssg + t_dec
 
-    # the same three calls without graph capture (direct C-ABI calls, device-resident inputs)
+    # the same call without graph capture (a direct C-ABI call, device-resident inputs)
     uevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps):
         flush_l2()
         uevs[i][0].record(stream)
-        for fn in calls[:3]:
-            fn()
+        calls[4]()
         uevs[i][1].record(stream)
     torch.cuda.synchronize()
     t_ssg_direct = float(np.mean([a.elapsed_time(b) for a, b in uevs]))
 
     # per-call breakdown (same flush between steps; separate graphs per call)
-    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     for i in range(args.steps):
         flush_l2()
         bevs[i][0].record(stream)
@@ -251,7 +251,7 @@ def run_ours(args):
             g.replay()
             bevs[i][j + 1].record(stream)
     torch.cuda.synchronize()
-    per = np.array([[bevs[i][j].elapsed_time(bevs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    per = np.array([[bevs[i][j].elapsed_time(bevs[i][j + 1]) for j in range(5)] for i in range(args.steps)])
     mean = per.mean(axis=0)
     t_ssg, t_step, t_dec = max_over_ranks([t_ssg, t_step, t_dec], dev)
     mean = np.array(max_over_ranks(list(mean), dev))
@@ -266,8 +266,8 @@ def run_ours(args):
     dec_gbs = decode_b / (t_dec * 1e-3) / 1e9
     # dominant call by time -> roofline object (all HBM-bound)
     calls = {"score": (mean[0], score_b), "select": (mean[1], 0), "gather": (mean[2], gather_b),
-             "decode": (mean[3], decode_b)}
-    dom = max(calls, key=lambda c: calls[c][0])
+             "decode": (mean[3], decode_b), "compress": (mean[4], score_b + gather_b)}
+    dom = max(("compress", "decode"), key=lambda c: calls[c][0])   # the kernels of the timed step
     dom_gbs = calls[dom][1] / (calls[dom][0] * 1e-3) / 1e9 if calls[dom][1] else 0.0
     traffic = load_traffic(dom)
 
@@ -286,8 +286,9 @@ def run_ours(args):
             "config": {"workload": cfg["name"], "n_h": n_h, "n_kv": n_kv, "d_h": d, "seq_len": S, "window": w,
                        "pool": cfg["pool_k"], "budget": B, "decode_batch": nb,
                        "l2": "flushed between steps (256 MiB write + 256 MiB read sweep, outside the timed events)",
-                       "launch": "score+select+gather as one CUDA graph (timed for value), decode as a second; "
-                                 "breakdown_us from one graph per call",
+                       "launch": "kvc_compress_window (score+select+gather in one call) as one CUDA graph, timed "
+                                 "for value; decode as a second graph; breakdown_us from one graph per call "
+                                 "(the three separate calls, decode and the one-call form)",
                        "parallelism": f"replicas x{world}"},
             "gbs": round(ssg_gbs, 1),
             "decode": {"gbs": round(dec_gbs, 1), "us": round(t_dec * 1e3, 2), "frac_of_8000": round(dec_gbs / 8000, 3)},
@@ -336,9 +337,7 @@ def run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, 
         d_k.copy_(h_k, non_blocking=True)
         d_v.copy_(h_v, non_blocking=True)
         qd.copy_(h_qd, non_blocking=True)
-        comp.score(d_q, d_k, stream)
-        comp.select(stream)
-        comp.gather(d_k, d_v, stream)
+        comp.compress(d_q, d_k, d_v, stream)
         dec.run(qd, kc_all, vc_all, off, ln, stream)
         h_idx.copy_(comp.buf.idx, non_blocking=True)
         h_out.copy_(dec.out, non_blocking=True)

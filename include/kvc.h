@@ -147,6 +147,28 @@ kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_hos
                             kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * kvc_compress_window: kvc_score_window, kvc_select_topk and kvc_gather_kv in
+ * one call, with the same arguments, layouts and results as the three calls
+ * in sequence (plus v, idx, k_out, v_out, budget and cu_budget of the latter
+ * two).  KVC_BF16 batches whose every (sequence, head, key chunk) work item
+ * fits on the GPU at once, with key chunks of at most 32768 keys, run it as
+ * ONE cooperative launch: after the pool, the CTAs of each (sequence, head)
+ * find the budgeted top-k together (a three-level radix select through small
+ * per-head histograms in the workspace) and each gathers the rows it kept.
+ * Other batches run the three calls.  ws: kvc_score_window_workspace_size()
+ * bytes, zeroed before its first use.  The pages define the three steps
+ * (SnapKV observation window, "Variantes de l'attention et compression du
+ * cache KV", section "Compresser un cache existant"); fusing them is this
+ * library's.
+ * ------------------------------------------------------------------------ */
+kvc_status kvc_compress_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host,
+                               const int32_t *cu_seqlens, const int32_t *cu_budget, int n_h, int n_kv,
+                               int d_h, int w, int pool_k, int budget, float scale, const void *q_win,
+                               const void *k, const void *v, float *scores, float *scores_raw,
+                               int32_t *idx, void *k_out, void *v_out, void *ws, size_t ws_bytes,
+                               kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Budgeted per-KV-head top-k (SnapKV keeps a chosen subset; the recent window
  * is always kept, as a sliding window keeps its recent region).
  *

@@ -68,7 +68,7 @@ struct ScorePlan {
   bool tc = false, fused = false;
   int R = 0, R_pad = 0, tile = 0, keys_per_chunk = 0, n_chunks = 0;
   Batch bt;
-  size_t off_sync = 0, off_part = 0, off_raw = 0, bytes = 0;
+  size_t off_sync = 0, off_hist = 0, off_cnt = 0, off_part = 0, off_raw = 0, bytes = 0;
 };
 
 kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w,
@@ -108,8 +108,11 @@ kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int
   pl->n_chunks = std::max(1, (pl->bt.max_len + pl->keys_per_chunk - 1) / pl->keys_per_chunk);
   // one cooperative launch when the whole grid is resident at once (one CTA per SM)
   pl->fused = pl->tc && (int64_t)n_kv * pl->n_chunks * n_seqs <= kvc::kNumSMs;
+  const size_t units = (size_t)n_seqs * n_kv;
   pl->off_sync = kErrWordBytes;
-  pl->off_part = round_up(pl->off_sync + (size_t)n_seqs * n_kv * 4 * sizeof(int), 256);
+  pl->off_hist = round_up(pl->off_sync + units * kvc::tc_counters_per_unit() * sizeof(int), 256);
+  pl->off_cnt = round_up(pl->off_hist + units * kvc::tc_hist_ints() * sizeof(int), 256);
+  pl->off_part = round_up(pl->off_cnt + units * pl->n_chunks * 2 * sizeof(int), 256);
   const size_t part_bytes = (size_t)n_seqs * n_kv * pl->n_chunks * pl->R_pad * sizeof(float2);
   pl->off_raw = round_up(pl->off_part + part_bytes, 256);
   pl->bytes = pl->off_raw + round_up((size_t)n_kv * pl->bt.T * sizeof(float), 256);
@@ -220,10 +223,29 @@ size_t kvc_score_window_workspace_size(kvc_dtype dt, int n_seqs, const int32_t *
   return pl.bytes;
 }
 
-kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
-                            int n_h, int n_kv, int d_h, int w, int pool_k, float scale, const void *q_win,
-                            const void *k, float *scores, float *scores_raw, void *ws, size_t ws_bytes,
-                            kvc_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// What kvc_compress_window adds to scoring: the selection and gather that run
+// inside the fused launch when it applies.
+struct SelectGather {
+  const int32_t *cu_budget;
+  int budget;
+  int total_budget;
+  int32_t *idx;
+  const void *v;
+  void *k_out, *v_out;
+};
+
+// Scoring (and, when sel != nullptr and the fused launch applies with every key
+// chunk small enough to keep on chip, the selection and gather too).  *done_sel
+// reports whether the selection and gather ran.
+kvc_status score_impl(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens, int n_h,
+                      int n_kv, int d_h, int w, int pool_k, float scale, const void *q_win, const void *k,
+                      float *scores, float *scores_raw, void *ws, size_t ws_bytes, kvc_stream_t stream,
+                      const SelectGather *sel, bool *done_sel) {
+  if (done_sel) *done_sel = false;
   ScorePlan pl;
   kvc_status s = plan_score(dt, n_seqs, seqlens_host, n_h, n_kv, d_h, w, &pl);
   if (s != KVC_OK) return s;
@@ -246,6 +268,8 @@ kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_hos
   a.raw = scores_raw ? scores_raw : reinterpret_cast<float *>(wsb + pl.off_raw);
   a.err = reinterpret_cast<int *>(wsb);
   a.sync = reinterpret_cast<int *>(wsb + pl.off_sync);
+  a.hist = reinterpret_cast<int *>(wsb + pl.off_hist);
+  a.cnt = reinterpret_cast<int *>(wsb + pl.off_cnt);
   a.scores = scores;
   a.pool_k = pool_k;
   a.fused = pl.fused;
@@ -253,12 +277,58 @@ kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_hos
   a.n_chunks = pl.n_chunks;
   a.keys_per_chunk = pl.keys_per_chunk;
   a.R_pad = pl.R_pad;
+  a.idx = nullptr; a.cu_budget = nullptr; a.v = nullptr; a.k_out = nullptr; a.v_out = nullptr;
+  a.total_budget = 0; a.budget = 0;
+  const bool fuse_sel = sel && pl.fused && pl.keys_per_chunk <= kvc::tc_select_max_keys(d_h);
+  if (fuse_sel) {
+    a.idx = sel->idx; a.cu_budget = sel->cu_budget; a.v = sel->v; a.k_out = sel->k_out; a.v_out = sel->v_out;
+    a.total_budget = sel->total_budget; a.budget = sel->budget;
+  }
   cudaError_t e = pl.tc ? kvc::score_window_tc(a, st) : kvc::score_window_simt(a, st);
   if (e != cudaSuccess) return cuda_fail(e, "score kernels");
+  if (done_sel) *done_sel = fuse_sel;
   if (pl.fused) return KVC_OK;   // the pool ran inside the fused launch
   e = kvc::pool_prefix(a.raw, scores, cu_seqlens, n_seqs, n_kv, a.T_total, pl.bt.max_len, w, pool_k, st);
   if (e != cudaSuccess) return cuda_fail(e, "pool kernel");
   return KVC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvc_status kvc_score_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                            int n_h, int n_kv, int d_h, int w, int pool_k, float scale, const void *q_win,
+                            const void *k, float *scores, float *scores_raw, void *ws, size_t ws_bytes,
+                            kvc_stream_t stream) {
+  return score_impl(dt, n_seqs, seqlens_host, cu_seqlens, n_h, n_kv, d_h, w, pool_k, scale, q_win, k, scores,
+                    scores_raw, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+kvc_status kvc_compress_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                               const int32_t *cu_budget, int n_h, int n_kv, int d_h, int w, int pool_k, int budget,
+                               float scale, const void *q_win, const void *k, const void *v, float *scores,
+                               float *scores_raw, int32_t *idx, void *k_out, void *v_out, void *ws, size_t ws_bytes,
+                               kvc_stream_t stream) {
+  // validate the selection and gather arguments before anything is launched
+  Batch bt;
+  kvc_status s = check_batch(n_seqs, seqlens_host, w, &bt);
+  if (s != KVC_OK) return s;
+  if (budget < w) return fail(KVC_ERR_INVALID_ARG, "budget (%d) must be >= w (%d): the window is always kept", budget, w);
+  if (!cu_budget) return fail(KVC_ERR_INVALID_ARG, "cu_budget is NULL");
+  if (!aligned16(idx) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out))
+    return fail(KVC_ERR_INVALID_ARG, "idx, v, k_out and v_out must be non-NULL and 16-byte aligned");
+  int64_t total = 0;
+  for (int b = 0; b < n_seqs; ++b) total += std::min(budget, seqlens_host[b]);
+  SelectGather sel{cu_budget, budget, (int)total, idx, v, k_out, v_out};
+  bool done = false;
+  s = score_impl(dt, n_seqs, seqlens_host, cu_seqlens, n_h, n_kv, d_h, w, pool_k, scale, q_win, k, scores,
+                 scores_raw, ws, ws_bytes, stream, &sel, &done);
+  if (s != KVC_OK || done) return s;
+  s = kvc_select_topk(n_seqs, seqlens_host, cu_seqlens, cu_budget, n_kv, w, budget, scores, idx, stream);
+  if (s != KVC_OK) return s;
+  return kvc_gather_kv(dt, n_seqs, seqlens_host, cu_seqlens, cu_budget, n_kv, d_h, budget, idx, k, v, k_out, v_out,
+                       stream);
 }
 
 kvc_status kvc_select_topk(int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,

@@ -22,10 +22,17 @@ struct ScoreArgs {
   float2 *part;          // [n_seqs, n_kv, n_chunks, R_pad] (m, l) per window row
   float *raw;            // [n_kv, T_total]
   float *scores;         // [n_kv, T_total] pooled (written by the fused path)
-  int *sync;             // fused path: 4 counters per (sequence, KV head), zero between calls
+  int *sync;             // fused path: counters per (sequence, KV head), zero between calls
   int *err;              // device error word (nonzero: a bounded wait gave up)
   int pool_k;
   bool fused;            // both passes and the pool in one cooperative launch
+  // selection and gather inside the fused launch (idx == nullptr: not requested)
+  int32_t *idx;
+  const int32_t *cu_budget;
+  const void *v;
+  void *k_out, *v_out;
+  int *hist, *cnt;
+  int total_budget, budget;
   int T_total;
   int n_chunks;          // key chunks per (sequence, KV head) in the launch grid
   int keys_per_chunk;    // multiple of the kernel's key tile
@@ -36,6 +43,9 @@ cudaError_t score_window_simt(const ScoreArgs &a, cudaStream_t st);
 cudaError_t score_window_tc(const ScoreArgs &a, cudaStream_t st);
 int simt_keys_per_tile();
 int tc_keys_per_tile();
+int tc_counters_per_unit();   // fused launch: arrival counters per (sequence, KV head)
+int tc_hist_ints();           // fused selection: histogram ints per (sequence, KV head)
+int tc_select_max_keys(int d_h);  // fused selection: largest key chunk it keeps on chip
 
 cudaError_t pool_prefix(const float *raw, float *scores, const int32_t *cu_seqlens, int n_seqs, int n_kv,
                         int T_total, int max_len, int w, int pool_k, cudaStream_t st);

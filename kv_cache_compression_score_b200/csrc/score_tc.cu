@@ -92,11 +92,25 @@ struct TcParams {
   float2 *part;
   float *raw;
   float *scores;   // fused path: pooled output
-  int *sync;       // fused path: 4 counters per (sequence, KV head), zero between calls
+  int *sync;       // fused path: kCtrPerUnit counters per (sequence, KV head), zero between calls
   int *err;
+  // fused selection and gather (idx == nullptr: the launch stops after the pool)
+  int32_t *idx;                 // [n_kv, total_budget]
+  const int32_t *cu_budget;
+  const uint8_t *v;             // V [T, n_kv, d_h]
+  uint8_t *k_out, *v_out;       // compact caches [total_budget, n_kv, d_h]
+  int *hist;                    // kHistInts per (sequence, KV head), zero between calls
+  int *cnt;                     // 2 per (sequence, KV head, key chunk)
+  int total_budget, budget;
   int n_h, n_kv, G, w, R, n_chunks, keys_per_chunk, T_total, pool_r;
   float c;   // scale * log2(e)
 };
+
+// fused selection: counters and per-(sequence, head) radix histograms
+constexpr int kCtrPerUnit = 8;     // stats, raw, depart, radix levels 1-3, counts, spare
+constexpr int kH1 = 4096, kH2 = 4096, kH3 = 256;
+constexpr int kHistInts = kH1 + kH2 + kH3;
+// keys of one chunk held in shared memory: the K ring (kStages tiles of kBN x d_h bf16) as uint32
 
 // Shared-memory objects of one CTA.
 struct TcSmem {
@@ -487,6 +501,222 @@ KVC_DEVINL void cta_teardown(const TcParams &p, const TcSmem &sm, uint32_t tmem_
   if (threadIdx.x == 0 && *sm.cta_err) atomicCAS(p.err, 0, 1);
 }
 
+// ----------------------------------------------------------- fused selection
+// Order-preserving 32-bit key of a float (larger float, larger key).
+KVC_DEVINL uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix sum of one int per thread (all kThreadsTC
+// threads call it); returns this thread's exclusive prefix, *total the sum.
+KVC_DEVINL int block_exclusive_scan(int v, int *scr, int *total) {
+  constexpr int kWarps = kThreadsTC / 32;
+  const int lane = lane_id(), warp = warp_id();
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scr[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < kWarps ? scr[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < kWarps) scr[32 + lane] = s;      // inclusive warp totals
+  }
+  __syncthreads();
+  const int base = warp > 0 ? scr[32 + warp - 1] : 0;
+  *total = scr[32 + kWarps - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// Scanning the bins of a global histogram from the top, the bin where the
+// running count reaches `need` (1 <= need <= total count) and the count in
+// the bins above it.  All threads call it and get the result.  Thread t holds
+// the 8 bins [nbins - 8 (t + 1), nbins - 8 t) in registers (two 16-byte
+// loads issued together), so the search costs one L2 round trip.
+KVC_DEVINL void find_bucket_from_top(const int *hist, int nbins, int need, int *scr, int &bin, int &above) {
+  const int t = threadIdx.x;
+  const bool mine = t < nbins / 8;
+  const int lo = nbins - 8 * (t + 1);
+  int h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (mine) {
+    const int4 a = __ldcg(reinterpret_cast<const int4 *>(hist + lo));
+    const int4 b = __ldcg(reinterpret_cast<const int4 *>(hist + lo) + 1);
+    h[0] = a.x; h[1] = a.y; h[2] = a.z; h[3] = a.w; h[4] = b.x; h[5] = b.y; h[6] = b.z; h[7] = b.w;
+  }
+  const int sum = ((h[0] + h[1]) + (h[2] + h[3])) + ((h[4] + h[5]) + (h[6] + h[7]));
+  int total;
+  const int before = block_exclusive_scan(sum, scr, &total);
+  if (mine && before < need && before + sum >= need) {
+    int run = before;
+#pragma unroll
+    for (int q = 7; q >= 0; --q) {
+      if (run + h[q] >= need) { scr[64] = lo + q; scr[65] = run; break; }
+      run += h[q];
+    }
+  }
+  __syncthreads();
+  bin = scr[64];
+  above = scr[65];
+  __syncthreads();
+}
+
+// After the pool, the CTAs of one (sequence, head) pick its budgeted top-k
+// (pooled prefix scores, lowest position first among equal scores, window
+// always kept, ascending positions) and gather the kept K/V rows.
+//   A three-level radix select on the order keys (12, 12 and 8 bits) finds
+//   the k-th largest key T and how many keys equal to T are taken: every CTA
+//   adds its histogram of the candidates to a per-head histogram in the
+//   workspace, waits on a counter, and reads the bucket holding the k-th key.
+//   (A single log-scale bucket with a candidate exchange was tried: pooled
+//   scores crowd into few buckets, so it was slower.)  Then every CTA
+//   publishes its counts of keys > T and == T, and writes its kept positions
+//   at (keys > T in earlier chunks) + (equal keys taken in earlier chunks) +
+//   its own rank, which gives the ascending order and the lowest-position tie
+//   rule across chunks.  The CTA gathers the rows it placed; the CTA holding
+//   position P writes and gathers the window.
+template <int D>
+KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const TcWork &wk, int *ctr, int nc,
+                                    const uint32_t *keys) {
+  const int tid = threadIdx.x;
+  const int P = wk.P, w = p.w;
+  const int kept = min(p.budget, wk.len);
+  const int k_sel = kept - w;                       // prefix tokens kept (the host checked budget >= w)
+  const int j0 = wk.key_begin;
+  const int n_my = max(0, min(wk.key_end, P) - j0);  // prefix keys of this chunk
+  const bool all = k_sel >= P;                      // the whole prefix is kept
+  int *scr = reinterpret_cast<int *>(sm.xch);        // scan scratch
+  int *sh = reinterpret_cast<int *>(sm.sq);          // shared histogram (the window block is free)
+  int *hist = p.hist + (size_t)(wk.b * p.n_kv + wk.h) * kHistInts;
+  int *cnt = p.cnt + (size_t)(wk.b * p.n_kv + wk.h) * p.n_chunks * 2;
+
+  uint32_t T = 0;
+  int need = 0;                                     // keys equal to T to take over the head
+  int base_gt = 0, base_eq = 0;                     // keys > T and == T in the earlier chunks
+  if (!all && k_sel > 0) {
+    uint32_t fixed = 0;                              // key bits fixed by the earlier levels
+    need = k_sel;
+    for (int lvl = 0; lvl < 3; ++lvl) {
+      const int nbins = lvl < 2 ? 4096 : 256;
+      const int shift = lvl == 0 ? 20 : (lvl == 1 ? 8 : 0);
+      int *gh = hist + (lvl == 0 ? 0 : (lvl == 1 ? kH1 : kH1 + kH2));
+      for (int b = tid; b < nbins; b += kThreadsTC) sh[b] = 0;
+      __syncthreads();
+      for (int i = tid; i < n_my; i += kThreadsTC) {
+        const uint32_t kk = keys[i];
+        const bool cand = lvl == 0 || (lvl == 1 ? (kk >> 20) == fixed : (kk >> 8) == fixed);
+        if (cand) atomicAdd(&sh[(kk >> shift) & (nbins - 1)], 1);
+      }
+      __syncthreads();
+      for (int b = tid; b < nbins; b += kThreadsTC)
+        if (sh[b]) atomicAdd(&gh[b], sh[b]);
+      __syncthreads();
+      if (tid == 0 && !arrive_and_wait(&ctr[3 + lvl], nc)) *sm.cta_err = 1;
+      __syncthreads();
+      int bin, above;
+      find_bucket_from_top(gh, nbins, need, scr, bin, above);
+      need -= above;
+      fixed = lvl == 0 ? (uint32_t)bin : (fixed << (lvl == 1 ? 12 : 8)) | (uint32_t)bin;
+    }
+    T = fixed;
+    // ---- counts of keys > T and == T per chunk, then the earlier chunks' sums
+    int gt = 0, eq = 0;
+    for (int i = tid; i < n_my; i += kThreadsTC) {
+      gt += keys[i] > T;
+      eq += keys[i] == T;
+    }
+    int tot_gt, tot_eq;
+    block_exclusive_scan(gt, scr, &tot_gt);
+    block_exclusive_scan(eq, scr, &tot_eq);
+    if (tid == 0) {
+      cnt[2 * wk.c] = tot_gt;
+      cnt[2 * wk.c + 1] = tot_eq;
+      if (!arrive_and_wait(&ctr[6], nc)) *sm.cta_err = 1;
+    }
+    __syncthreads();
+    int2 c2 = make_int2(0, 0);
+    for (int cc = tid; cc < wk.c; cc += kThreadsTC) {
+      const int2 v = __ldcg(reinterpret_cast<const int2 *>(cnt) + cc);
+      c2.x += v.x;
+      c2.y += v.y;
+    }
+    block_exclusive_scan(c2.x, scr, &base_gt);
+    block_exclusive_scan(c2.y, scr, &base_eq);
+  }
+
+  // ---- this chunk's output offset and its share of the equal keys
+  int off = 0, eq_take = 0;
+  if (all) {
+    off = j0;                                       // the kept prefix is the identity
+  } else if (k_sel > 0) {
+    off = base_gt + min(need, base_eq);
+    eq_take = max(0, need - base_eq);
+  }
+
+  // ---- ordered compaction: thread t walks a contiguous run of the chunk
+  const int total = p.total_budget;
+  const int cb = p.cu_budget[wk.b];
+  int32_t *idx = p.idx + (size_t)wk.h * total + cb;
+  int n_sel = 0;
+  if (all || k_sel > 0) {
+    const int run = (n_my + kThreadsTC - 1) / kThreadsTC;
+    const int i0 = min(n_my, tid * run), i1 = min(n_my, i0 + run);
+    int my_gt = 0, my_eq = 0;
+    if (!all)
+      for (int i = i0; i < i1; ++i) { my_gt += keys[i] > T; my_eq += keys[i] == T; }
+    int tot_gt, tot_eq;
+    int gt_b = block_exclusive_scan(all ? i1 - i0 : my_gt, scr, &tot_gt);
+    int eq_b = block_exclusive_scan(my_eq, scr, &tot_eq);
+    // (slot checks only matter if a bounded wait gave up and the counts are inconsistent)
+    auto put = [&](int slot, int pos) { if (slot >= 0 && slot < k_sel) idx[slot] = pos; };
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t kk = keys[i];
+      if (all || kk > T) {
+        put(off + gt_b + min(eq_b, eq_take), j0 + i);
+        ++gt_b;
+      } else if (kk == T) {
+        if (eq_b < eq_take) put(off + gt_b + eq_b, j0 + i);
+        ++eq_b;
+      }
+    }
+    n_sel = max(0, min(tot_gt + min(tot_eq, eq_take), k_sel - off));
+  }
+  // the window: positions P .. len-1 at slots k_sel .. kept-1, by the CTA holding P
+  const bool win_owner = wk.key_begin <= P && P < wk.key_end;
+  if (win_owner)
+    for (int t = tid; t < w; t += kThreadsTC) idx[k_sel + t] = P + t;
+  __syncthreads();
+
+  // ---- gather the rows this CTA placed (their slots are contiguous)
+  constexpr int kVec = D * 2 / 16;                  // 16-byte vectors per head row (bf16)
+  const size_t head_bytes = (size_t)D * 2;
+  auto gather_slots = [&](int s0, int n) {
+    for (int e = tid; e < n * kVec; e += kThreadsTC) {
+      const int slot = s0 + e / kVec, c = e % kVec;
+      const int pos = __ldcg(idx + slot);
+      const size_t dst = ((size_t)(cb + slot) * p.n_kv + wk.h) * head_bytes + (size_t)c * 16;
+      uint4 kv_k = make_uint4(0, 0, 0, 0), kv_v = make_uint4(0, 0, 0, 0);
+      if (pos >= 0 && pos < wk.len) {            // a position outside the sequence gives a zero row
+        const size_t src = ((size_t)(wk.t0 + pos) * p.n_kv + wk.h) * head_bytes + (size_t)c * 16;
+        kv_k = ld_stream16(reinterpret_cast<const uint8_t *>(p.k) + src);
+        kv_v = ld_stream16(p.v + src);
+      }
+      st_stream16(p.k_out + dst, kv_k);
+      st_stream16(p.v_out + dst, kv_v);
+    }
+  };
+  if (off >= 0) gather_slots(off, n_sel);
+  if (win_owner) gather_slots(k_sel, w);
+}
+
 // One pass per launch (the grid does not fit on the GPU at once).
 template <int D, bool kScorePass>
 __global__ void __launch_bounds__(kThreadsTC, 1)
@@ -512,7 +742,7 @@ score_fused_kernel(TcParams p) {
   const TcSmem sm = carve_smem<D>(smem_raw);
   const uint32_t tmem_base = cta_setup<D>(p, sm, wk);
   const int nc = (wk.len + p.keys_per_chunk - 1) / p.keys_per_chunk;
-  int *ctr = p.sync + (size_t)(wk.b * p.n_kv + wk.h) * 4;
+  int *ctr = p.sync + (size_t)(wk.b * p.n_kv + wk.h) * kCtrPerUnit;
 
   tc_pass<D, false>(p, sm, wk, tmem_base, false);
 
@@ -537,21 +767,54 @@ score_fused_kernel(TcParams p) {
   {
     const float *src = p.raw + (size_t)wk.h * p.T_total + wk.t0;
     float *dst = p.scores + (size_t)wk.h * p.T_total + wk.t0;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(sm.sk);   // the K ring is no longer needed
     const int r = p.pool_r;
+    // stage the chunk's raw scores and the halo in the (free) window-block
+    // area with coalesced loads; neighbours outside the prefix read as -inf
+    float *stage = reinterpret_cast<float *>(sm.sq);
+    const int s_lo = wk.key_begin - r, s_n = min(wk.key_end, wk.P) + r - s_lo;
+    const bool staged = s_n <= TcLayout<D>::kQBytes / 4;
+    if (staged) {
+      for (int e = threadIdx.x; e < s_n; e += kThreadsTC) {
+        const int j = s_lo + e;
+        stage[e] = (j >= 0 && j < wk.P) ? __ldcg(src + j) : kNegInf;
+      }
+      __syncthreads();
+    }
     for (int j = wk.key_begin + threadIdx.x; j < wk.key_end; j += kThreadsTC) {
       float v = kPosInf;
       if (j < wk.P) {
-        const int lo = max(0, j - r), hi = min(wk.P - 1, j + r);
-        v = __ldcg(src + lo);
-        for (int q = lo + 1; q <= hi; ++q) v = fmaxf(v, __ldcg(src + q));
+        if (staged) {
+          const float *c = stage + (j - s_lo);
+          v = c[0];
+          for (int q = 1; q <= r; ++q) v = fmaxf(v, fmaxf(c[-q], c[q]));
+        } else {
+          const int lo = max(0, j - r), hi = min(wk.P - 1, j + r);
+          v = __ldcg(src + lo);
+          for (int q = lo + 1; q <= hi; ++q) v = fmaxf(v, __ldcg(src + q));
+        }
+        if (p.idx) keys[j - wk.key_begin] = order_key(v);
       }
       dst[j] = v;
     }
   }
+  if (p.idx) {
+    __syncthreads();
+    fused_select_gather<D>(p, sm, wk, ctr, nc, reinterpret_cast<const uint32_t *>(sm.sk));
+  }
 
-  // the last CTA of this head to leave resets the counters for the next call
+  // the last CTA of this head to leave resets the counters (and histograms)
+  // for the next call
   __syncthreads();
-  if (threadIdx.x == 0 && atomicAdd(&ctr[2], 1) == nc - 1) { ctr[0] = 0; ctr[1] = 0; ctr[2] = 0; }
+  if (threadIdx.x == 0) sm.off[0] = __int_as_float(atomicAdd(&ctr[2], 1) == nc - 1 ? 1 : 0);
+  __syncthreads();
+  if (__float_as_int(sm.off[0])) {
+    if (p.idx) {
+      int *hist = p.hist + (size_t)(wk.b * p.n_kv + wk.h) * kHistInts;
+      for (int e = threadIdx.x; e < kHistInts; e += kThreadsTC) hist[e] = 0;
+    }
+    if (threadIdx.x < kCtrPerUnit) ctr[threadIdx.x] = 0;
+  }
   cta_teardown(p, sm, tmem_base);
 }
 
@@ -566,6 +829,15 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
   p.scores = a.scores;
   p.sync = a.sync;
   p.err = a.err;
+  p.idx = a.fused ? a.idx : nullptr;
+  p.cu_budget = a.cu_budget;
+  p.v = static_cast<const uint8_t *>(a.v);
+  p.k_out = static_cast<uint8_t *>(a.k_out);
+  p.v_out = static_cast<uint8_t *>(a.v_out);
+  p.hist = a.hist;
+  p.cnt = a.cnt;
+  p.total_budget = a.total_budget;
+  p.budget = a.budget;
   p.n_h = a.n_h; p.n_kv = a.n_kv; p.G = a.n_h / a.n_kv; p.w = a.w; p.R = p.G * a.w;
   p.n_chunks = a.n_chunks; p.keys_per_chunk = a.keys_per_chunk; p.T_total = a.T_total;
   p.pool_r = a.pool_k / 2;
@@ -601,6 +873,9 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
 }  // namespace
 
 int tc_keys_per_tile() { return kBN; }
+int tc_counters_per_unit() { return kCtrPerUnit; }
+int tc_hist_ints() { return kHistInts; }
+int tc_select_max_keys(int d_h) { return kStages * kBN * d_h * 2 / 4; }
 
 cudaError_t score_window_tc(const ScoreArgs &a, cudaStream_t st) {
   if (a.d_h == 64) return launch_tc<64>(a, st);

@@ -34,6 +34,9 @@ SIGNATURES = {
     "kvc_score_window_workspace_size": (_c_sz, [_c_int, _c_int, _c_p, _c_int, _c_int, _c_int, _c_int]),
     "kvc_score_window": (_c_int, [_c_int, _c_int, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_f,
                                   _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "kvc_compress_window": (_c_int, [_c_int, _c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_int, _c_f, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz,
+                                     _c_p]),
     "kvc_select_topk": (_c_int, [_c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p]),
     "kvc_gather_kv": (_c_int, [_c_int, _c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p,
                                _c_p, _c_p, _c_p]),
@@ -157,6 +160,16 @@ def kvc_score_window(q_win, k, seqlens, cu_seqlens, n_h: int, n_kv: int, w: int,
     _check(lib().kvc_score_window(dtype_code(k), len(sl), p, _dptr(cu_seqlens), n_h, n_kv, k.shape[-1], w, pool_k,
                                   scale, _dptr(q_win), _dptr(k), _dptr(scores), _dptr(scores_raw), _dptr(ws),
                                   ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def kvc_compress_window(q_win, k, v, seqlens, cu_seqlens, cu_budget, n_h: int, n_kv: int, w: int, pool_k: int,
+                        budget: int, scale: float, scores, scores_raw, idx, k_out, v_out, ws, stream=None) -> None:
+    """Score, select and gather in one call (one launch where the fused path applies)."""
+    sl, p = _host_i32(seqlens)
+    _check(lib().kvc_compress_window(dtype_code(k), len(sl), p, _dptr(cu_seqlens), _dptr(cu_budget), n_h, n_kv,
+                                     k.shape[-1], w, pool_k, budget, scale, _dptr(q_win), _dptr(k), _dptr(v),
+                                     _dptr(scores), _dptr(scores_raw), _dptr(idx), _dptr(k_out), _dptr(v_out),
+                                     _dptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def kvc_select_topk(seqlens, cu_seqlens, cu_budget, n_kv: int, w: int, budget: int, scores, idx,

@@ -98,6 +98,14 @@ class Compressor:
         b = self.buf
         kvc.kvc_gather_kv(b.seqlens, b.cu_seqlens, b.cu_budget, self.budget, b.idx, k, v, b.k_c, b.v_c, stream)
 
+    def compress(self, q_win, k, v, stream=None):
+        """kvc_compress_window: the same three steps in one call."""
+        b = self.buf
+        kvc.kvc_compress_window(q_win, k, v, b.seqlens, b.cu_seqlens, b.cu_budget, self.n_h, self.n_kv, self.w,
+                                self.pool_k, self.budget, self.scale, b.scores, b.scores_raw, b.idx, b.k_c, b.v_c,
+                                b.ws, stream)
+        return b.idx, b.k_c, b.v_c
+
     def run(self, q_win, k, v, stream=None):
         self.score(q_win, k, stream)
         self.select(stream)

@@ -73,7 +73,7 @@ def upload_batch(bt, dtype):
 
 
 def run_and_check_compress(dtype, lengths, n_h, n_kv, d, w, pool_k, budget, seed, boost_frac=0.0, boost=3.0,
-                           check_gather=True, repeat=1):
+                           check_gather=True, repeat=1, fused_call=False):
     """Whole score -> select -> gather path on one seeded batch, every output
     compared with the oracle (after `repeat` runs on the same buffers).
     Returns a dict of the pieces for further checks."""
@@ -81,11 +81,14 @@ def run_and_check_compress(dtype, lengths, n_h, n_kv, d, w, pool_k, budget, seed
     q, k, v = upload_batch(bt, dtype)
     comp = Compressor(dtype, lengths, n_h, n_kv, d, w, pool_k, budget)
     for _ in range(repeat):
-        comp.run(q, k, v)
+        if fused_call:
+            comp.compress(q, k, v)
+        else:
+            comp.run(q, k, v)
     torch.cuda.synchronize()
     assert comp.device_error_word() == 0
     # the per-(sequence, head) arrival counters are left at zero for the next call
-    ctr = comp.buf.ws[256:256 + 16 * len(lengths) * n_kv].view(torch.int32)
+    ctr = comp.buf.ws[256:256 + 32 * len(lengths) * n_kv].view(torch.int32)
     assert int(ctr.abs().sum().item()) == 0
     cu = bt["cu_seqlens"]
     raw_o = O.raw_scores(bt["q_win"], bt["k"], cu, n_h, n_kv, w, dtype)

@@ -32,8 +32,11 @@ def _built():
     assert torch.cuda.is_available()
 
 
-def test_llama8b_layer_s32k():
-    r = run_and_check_compress("bf16", [32768], N_H, N_KV, D, W, POOL, 2048, seed=1002, boost_frac=0.01)
+@pytest.mark.parametrize("fused", [False, True])
+def test_llama8b_layer_s32k(fused):
+    """fused: kvc_compress_window (one launch: score, select and gather)."""
+    r = run_and_check_compress("bf16", [32768], N_H, N_KV, D, W, POOL, 2048, seed=1002, boost_frac=0.01,
+                               fused_call=fused)
     # decode at batch 16 over 16 compact caches of 2048 rows (the step's own cache first)
     kc = [from_device(r["comp"].buf.k_c)]
     vc = [from_device(r["comp"].buf.v_c)]
@@ -45,10 +48,11 @@ def test_llama8b_layer_s32k():
     run_and_check_decode("bf16", q, np.concatenate(kc), np.concatenate(vc), np.arange(16) * 2048, [2048] * 16, N_KV)
 
 
-@pytest.mark.parametrize("budget", [4096, 131072])
-def test_long_context_s128k(budget):
+@pytest.mark.parametrize("budget,fused", [(4096, False), (131072, False), (4096, True), (131072, True)])
+def test_long_context_s128k(budget, fused):
     S = 131072
-    r = run_and_check_compress("bf16", [S], N_H, N_KV, D, W, POOL, budget, seed=1003, boost_frac=0.01)
+    r = run_and_check_compress("bf16", [S], N_H, N_KV, D, W, POOL, budget, seed=1003, boost_frac=0.01,
+                               fused_call=fused)
     if budget >= S:
         # identity: every position kept, compact cache == cache, decode == full attention
         np.testing.assert_array_equal(r["idx_g"], np.broadcast_to(np.arange(S), (N_KV, S)))
@@ -83,9 +87,11 @@ def test_fastkv_tsp_layer_and_next_layer():
     run_and_check_compress("bf16", [k_tsp + W], N_H, N_KV, D, W, POOL, kv_budget, seed=1004 + 16, boost_frac=0.01)
 
 
-def test_ragged_16_sequences():
+@pytest.mark.parametrize("fused", [False, True])
+def test_ragged_16_sequences(fused):
     lens = synth.ragged_lengths(1005, 16, 4096, 65536)
-    r = run_and_check_compress("bf16", lens, N_H, N_KV, D, W, POOL, 1024, seed=1005, boost_frac=0.01)
+    r = run_and_check_compress("bf16", lens, N_H, N_KV, D, W, POOL, 1024, seed=1005, boost_frac=0.01,
+                               fused_call=fused)
     cb = O.budget_offsets(lens, 1024)
     q = synth.decode_queries(1013, 16, N_H, D, "bf16")
     run_and_check_decode("bf16", q, from_device(r["comp"].buf.k_c), from_device(r["comp"].buf.v_c), cb[:-1],

@@ -73,7 +73,7 @@ def test_fused_wait_gives_up_and_reports():
     bt = synth.packed_batch(4246, lengths, 32, 8, 128, 32, "bf16", 0.0, 3.0)
     q, k, v = (to_device(bt[x], "bf16") for x in ("q_win", "k", "v"))
     comp = Compressor("bf16", lengths, 32, 8, 128, 32, 7, 200)
-    ctr = comp.buf.ws[256:256 + 16 * 8].view(torch.int32)
+    ctr = comp.buf.ws[256:256 + 32 * 8].view(torch.int32)
     ctr[0] = -1 << 20                                   # head 0's stats barrier can never fill
     comp.score(q, k)
     assert kvc.kvc_check_workspace(comp.buf.ws) == kvc.KVC_ERR_DEVICE_CHECK
@@ -83,6 +83,57 @@ def test_fused_wait_gives_up_and_reports():
     assert kvc.kvc_check_workspace(comp.buf.ws) == kvc.KVC_OK
     raw_o = O.raw_scores(bt["q_win"], bt["k"], bt["cu_seqlens"], 32, 8, 32, "bf16")
     assert_scores_close(comp.buf.scores_raw.cpu().numpy(), raw_o, what="raw scores after recovery")
+
+
+@pytest.mark.parametrize("lengths,budget", [([3000, 1500], 300), ([4097], 1000), ([700, 64], 700), ([700, 64], 32),
+                                            ([1000, 300, 129, 32, 777], 200)])
+def test_compress_window_fused_select_gather(lengths, budget):
+    """kvc_compress_window: scores, indices and gathered rows against the
+    oracle (one launch with selection inside where it applies; the identity,
+    budget == window and tiny-sequence edges included)."""
+    run_and_check_compress("bf16", lengths, 32, 8, 128, 32, 7, budget, seed=4250, fused_call=True, repeat=2)
+
+
+def test_compress_window_ties_exact():
+    """Many equal pooled scores (boost-free keys, pool 7 plateaus): the fused
+    selection keeps the lowest positions among equal scores, checked against
+    the oracle's exact rule; repeated calls reuse the workspace."""
+    r = run_and_check_compress("bf16", [2500], 32, 8, 128, 32, 7, 600, seed=4251, fused_call=True, repeat=3,
+                               boost_frac=0.01, boost=40.0)
+    # on the GPU's own fp32 pooled scores the selection is exact: identical to
+    # the oracle's rule applied to those same values
+    pooled_g = r["comp"].buf.scores.cpu().numpy().astype(np.float64)
+    idx_ref = O.select_topk(pooled_g, r["bt"]["cu_seqlens"], 32, 600)
+    assert np.array_equal(r["idx_g"], idx_ref)
+
+
+def test_compress_window_all_equal_scores_overflow_path():
+    """K = 0: every pooled prefix score is equal, so the bucket of the k-th key
+    holds the whole prefix (more candidates than the exchange takes) and the
+    radix path decides; the lowest positions must be kept, exactly as the
+    oracle's rule (and the tie-break pin) says."""
+    lengths, budget = [5000, 3000], 1000
+    bt = synth.packed_batch(4254, lengths, 32, 8, 128, 32, "bf16", 0.0, 3.0)
+    q, v = to_device(bt["q_win"], "bf16"), to_device(bt["v"], "bf16")
+    k = torch.zeros_like(v)
+    comp = Compressor("bf16", lengths, 32, 8, 128, 32, 7, budget)
+    for _ in range(2):
+        comp.compress(q, k, v)
+    torch.cuda.synchronize()
+    assert comp.device_error_word() == 0
+    cu = bt["cu_seqlens"]
+    idx_o = O.select_topk(O.pool_prefix(O.raw_scores(bt["q_win"], np.zeros_like(bt["k"]), cu, 32, 8, 32, "bf16"),
+                                        cu, 32, 7), cu, 32, budget)
+    assert np.array_equal(comp.buf.idx.cpu().numpy(), idx_o)
+    for b, L in enumerate(lengths):
+        seg = comp.buf.idx.cpu().numpy()[:, b * budget:(b + 1) * budget]
+        assert np.array_equal(seg, np.broadcast_to(np.r_[np.arange(budget - 32), np.arange(L - 32, L)], seg.shape))
+
+
+def test_compress_window_split_fallback():
+    """More work items than fit at once: kvc_compress_window runs the three calls."""
+    lengths = synth.ragged_lengths(4252, 20, 40, 700).tolist()
+    run_and_check_compress("bf16", lengths, 32, 8, 128, 32, 7, 96, seed=4253, fused_call=True)
 
 
 def test_bf16_tensor_core_small_block_d64():
