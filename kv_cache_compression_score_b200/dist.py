@@ -42,3 +42,20 @@ def max_over_ranks(values, device=None):
 def whole_job_rate(units_per_rank: float, world: int, max_time_s: float) -> float:
     """Aggregate throughput: the units all ranks processed over the slowest rank's time."""
     return world * float(units_per_rank) / float(max_time_s)
+
+
+def tsp_exchange_raw(raw_local: torch.Tensor, group=None) -> torch.Tensor:
+    """The one exchange step of head-sharded token-selective propagation
+    (FastKV section 2.A: saliency aggregated over all heads of the layer).
+
+    raw_local is this rank's [n_local, S] float32 raw window scores (its KV
+    heads; every rank holds the same n_local).  It is summed element-wise
+    over the ranks in place (all-reduce, SUM) and returned: the TSP step then
+    adds its n_local rows, which gives the sum over every head of the layer,
+    and every rank selects the same token set.  Without a process group the
+    tensor is returned unchanged.  The addition order differs from one
+    device's, so equal-up-to-rounding scores may tie-break differently (the
+    selection agrees outside the 1e-5 tie band)."""
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(raw_local, op=dist.ReduceOp.SUM, group=group)
+    return raw_local

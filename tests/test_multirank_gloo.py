@@ -50,6 +50,38 @@ def test_two_ranks_gloo():
     assert kd.whole_job_rate(32768, world, 2.0) == 32768.0
 
 
+def _tsp_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import torch
+        from oracle import kvc_oracle as O
+        S, w, n_kv = 600, 32, 8
+        raw = synth.random_scores(1234, (n_kv, S), 0)           # the same full [8, S] on every rank
+        n_local = n_kv // world
+        mine = torch.from_numpy(np.ascontiguousarray(raw[rank * n_local:(rank + 1) * n_local], dtype=np.float32))
+        red = kd.tsp_exchange_raw(mine)
+        idx = O.tsp_select(red.numpy().astype(np.float64), S, w, 7, 100)
+        out[rank] = idx.tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tsp_head_sharded_exchange():
+    """Head-sharded TSP over 2 gloo ranks: after the all-reduce of the raw rows
+    every rank selects the token set the unsharded layer selects."""
+    from oracle import kvc_oracle as O
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_tsp_worker, args=(world, port, out), nprocs=world, join=True)
+    raw = synth.random_scores(1234, (8, 600), 0).astype(np.float32).astype(np.float64)
+    ref = O.tsp_select(raw, 600, 32, 7, 100)
+    assert out[0] == out[1] == ref.tolist()
+
+
 def test_shard_cover_exactly_once():
     for n in (0, 1, 7, 16, 101):
         for world in (1, 2, 3, 8):
