@@ -1,8 +1,8 @@
 """Plain fp64 CPU oracle for observation-window KV-cache compression.
 
 TEST INFRASTRUCTURE.  Only the test-suite, the package smoke check and the
-bench's CPU-baseline leg may import this module.  The CUDA library never calls
-it and shares no code with it.
+bench's CPU-baseline and reference legs may import this module.  The CUDA
+library never calls it and shares no code with it.
 
 What it computes, step by step, in float64 from the stored inputs (fp32 values
 or bf16 bit patterns, both widened exactly):
@@ -32,6 +32,11 @@ or bf16 bit patterns, both widened exactly):
    of k_tsp prefix positions plus the window, hidden rows copied.
 8. ``cache_bytes`` -- 2 * L * S * n_kv * d_h * b (attention-variants page,
    section "MHA et GQA").
+
+Every function above is pinned by tests/test_oracle_pins.py (closed forms,
+invariants, the pages' worked cache-size example, brute force on tiny inputs,
+library cross-checks).  The readings below are choices, not facts from the
+pages: parity is unpinned for them.
 
 Readings of points the pages leave open (each also listed in the design doc):
 * logit scale: passed explicitly, 1/sqrt(d_h) by default;
