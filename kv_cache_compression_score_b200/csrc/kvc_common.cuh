@@ -80,7 +80,6 @@ KVC_DEVINL void allow_dependents() { asm volatile("griddepcontrol.launch_depende
 // that runs past its time limit returns false; the caller records an error
 // code, stops issuing work and leaves through its normal exit path.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kSpinLimit = 1u << 22;          // iteration bound of plain polling loops
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s; healthy waits take microseconds
 constexpr uint32_t kSuspendHintNs = 1000000;       // a try_wait may sleep up to this long
 

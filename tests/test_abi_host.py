@@ -137,3 +137,28 @@ def test_check_workspace_and_launch_count_need_no_gpu_to_validate(L):
     assert e.value.status == kvc.KVC_ERR_INVALID_ARG
     assert L.kvc_status_string(kvc.KVC_ERR_DEVICE_CHECK) == b"KVC_ERR_DEVICE_CHECK"
     assert kvc.kvc_launch_count() >= 0
+
+
+def test_compress_window_rejects_before_launch(L):
+    """kvc_compress_window validates the selection and gather arguments as well
+    as the scoring ones, before anything is launched."""
+    sl = np.array([300, 100], np.int32)
+    slp = sl.ctypes.data_as(ctypes.c_void_p)
+    ws_ok = kvc.kvc_score_window_workspace_size(kvc.KVC_BF16, sl, 32, 8, 128, 32)
+    assert ws_ok > 0
+
+    def call(budget=64, cu_budget=P16, v=P16, idx=P16, k_out=P16, v_out=P16, ws_bytes=ws_ok, pool_k=7, w=32,
+             dt=kvc.KVC_BF16):
+        return L.kvc_compress_window(dt, 2, slp, P16, cu_budget, 32, 8, 128, w, pool_k, budget, 0.0, P16, P16, v,
+                                     P16, None, idx, k_out, v_out, P16, ws_bytes, None)
+
+    assert call(budget=31) == INVALID and b"window" in L.kvc_last_error()
+    assert call(cu_budget=None) == INVALID
+    assert call(v=None) == INVALID
+    assert call(idx=P8) == INVALID
+    assert call(k_out=None) == INVALID
+    assert call(v_out=P8) == INVALID
+    assert call(pool_k=6) == INVALID
+    assert call(w=101) == INVALID                        # the second sequence is shorter than the window
+    assert call(ws_bytes=64) == WORKSPACE
+    assert call(dt=5) == UNSUPPORTED
