@@ -1,6 +1,6 @@
 """Benchmark of the observation-window KV-compression hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = one pass of the whole path over one batch of seeded synthetic input
 (Llama-3-8B-shaped layer: n_h 32, n_kv 8, d_h 128, bf16, S 32768, window 32,
@@ -39,7 +39,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-CONFIG2 = dict(name="llama3-8b-layer-S32768-B2048", n_h=32, n_kv=8, d_h=128, S=32768, w=32, pool_k=7, budget=2048,
+LLAMA3_8B_S32K = dict(name="llama3-8b-layer-S32768-B2048", n_h=32, n_kv=8, d_h=128, S=32768, w=32, pool_k=7, budget=2048,
                decode_batch=16, boost_frac=0.01, boost=3.0, seed=1002, dtype="bf16")
 METRIC = "score+select+gather K-tok/s & GB/s at S=32K; decode-attn GB/s vs 8 TB/s HBM"
 FALLBACK_HBM_GBS = 6650.0
@@ -137,7 +137,7 @@ def run_ours(args):
     from kv_cache_compression_score_b200.dist import max_over_ranks, rank_seed
     from kv_cache_compression_score_b200.runner import Compressor, Decoder, to_device
 
-    cfg = dict(CONFIG2)
+    cfg = dict(LLAMA3_8B_S32K)
     seed = rank_seed(cfg["seed"], rank)
     S, n_h, n_kv, d, w, B, nb = cfg["S"], cfg["n_h"], cfg["n_kv"], cfg["d_h"], cfg["w"], cfg["budget"], \
         cfg["decode_batch"]
@@ -404,7 +404,7 @@ def run_reference(args):
     if rank != 0:
         return
     from kv_cache_compression_score_b200 import synth
-    cfg = dict(CONFIG2)
+    cfg = dict(LLAMA3_8B_S32K)
     bt = synth.packed_batch(cfg["seed"], [cfg["S"]], cfg["n_h"], cfg["n_kv"], cfg["d_h"], cfg["w"], cfg["dtype"],
                             cfg["boost_frac"], cfg["boost"])
     for _ in range(args.warmup):

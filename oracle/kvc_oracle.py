@@ -38,7 +38,7 @@ invariants, the pages' worked cache-size example, brute force on tiny inputs,
 library cross-checks).  The readings below are choices, not facts from the
 pages: parity is unpinned for them.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
 * logit scale: passed explicitly, 1/sqrt(d_h) by default;
 * GQA mapping: query head qh uses KV head qh // G (contiguous groups);
 * softmax domain: the whole visible row, window keys included; only prefix

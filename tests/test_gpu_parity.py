@@ -24,7 +24,7 @@ def _built():
 
 
 # ------------------------------------------------------------------ scoring
-def test_config1_fp32_whole_path():
+def test_small_fp32_layer_s2048_whole_path():
     """One layer, n_h 4, n_kv 2, d_h 64, S 2048, fp32, w 32, pool 7, B 256."""
     r = run_and_check_compress("f32", [2048], 4, 2, 64, 32, 7, 256, seed=1001)
     assert r["n_diff"] == 0
