@@ -256,6 +256,30 @@ def run_ours(args):
     t_ssg, t_step, t_dec = max_over_ranks([t_ssg, t_step, t_dec], dev)
     mean = np.array(max_over_ranks(list(mean), dev))
 
+    # ---- FastKV token-selective propagation on the same layer size (timed on
+    # its own, not part of the step): head-summed pooled scores of 8 heads,
+    # k_tsp = floor(0.2 S) tokens plus the window, bf16 hidden rows [S, 4096]
+    from kv_cache_compression_score_b200.runner import TspSelector
+    k_tsp, d_hidden = (S * 2) // 10, 4096
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed + 11)
+    hidden = torch.randn((S, d_hidden), generator=gen, device=dev).to(torch.bfloat16)
+    raw_tsp = torch.from_numpy(synth.random_scores(seed + 12, (n_kv, S))).to(dev)
+    tsp = TspSelector(S, w, cfg["pool_k"], k_tsp, d_hidden, "bf16", device=dev)
+    tsp.run(raw_tsp, hidden)
+    torch.cuda.synchronize()
+    g_tsp, _ = capture([lambda: tsp.run(raw_tsp, hidden)])
+    tevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2()
+        tevs[i][0].record(stream)
+        g_tsp.replay()
+        tevs[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_tsp = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in tevs]))], dev)[0]
+    tsp_bytes = n_kv * S * 4 + 2 * (k_tsp + w) * d_hidden * 2   # raw scores read; hidden rows read and written
+    del hidden
+
     # ---- e2e: the same path through the C ABI with pinned host buffers
     e2e = run_e2e(args, cfg, bt, comp, dec, qd, off, ln, kc_all, vc_all, dev, stream, flush_l2)
     e2e["t_ms"] = max_over_ranks([e2e["t_ms"]], dev)[0]
@@ -298,6 +322,9 @@ def run_ours(args):
                              "graph_min": round(float(np.min(ssg_samples)) * 1e3, 2),
                              "uncaptured_mean": round(t_ssg_direct * 1e3, 2)},
             "ssg_frac_of_8000": round(ssg_gbs / 8000, 3),
+            "tsp": {"us": round(t_tsp * 1e3, 2), "k_tsp": k_tsp, "hidden": [S, d_hidden],
+                    "gbs": round(tsp_bytes / (t_tsp * 1e-3) / 1e9, 1),
+                    "frac_of_measured_peak": round(tsp_bytes / (t_tsp * 1e-3) / 1e9 / hbm, 3)},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(dom_gbs, 1), "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom_gbs / hbm, 3),
                          "traffic": traffic},
