@@ -99,10 +99,6 @@ KVC_DEVINL void mbar_arrive(uint64_t *bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}"
                :: "r"(smem_u32(bar)) : "memory");
 }
-KVC_DEVINL void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-               :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
 // One wait step: the thread sleeps in hardware until the phase with the given
 // parity completes (returns true) or the suspend hint runs out (false), so a
 // waiting warp takes no issue slots from the warps doing the work.
@@ -121,21 +117,6 @@ KVC_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity))
     if (global_ns() - t0 > kWaitLimitNs) return false;
   return true;
-}
-
-// ---------------------------------------------------------------------------
-// TMA (bulk tensor copies, no multicast) -- global -> shared, completion on an
-// mbarrier with a transaction byte count.
-// ---------------------------------------------------------------------------
-KVC_DEVINL void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar, int c0, int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];"
-      :: "r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-KVC_DEVINL void tma_prefetch_desc(const void *tmap) {
-  asm volatile("prefetch.tensormap [%0];" :: "l"(tmap) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -164,25 +145,6 @@ KVC_DEVINL void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uin
 KVC_DEVINL void umma_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                :: "r"(smem_u32(bar)) : "memory");
-}
-KVC_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane
-// (base + i), columns col .. col+31.
-KVC_DEVINL void tmem_ld32(uint32_t taddr, float *v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 32 lanes x 16 consecutive 32-bit columns, raw bits.  The registers hold the
