@@ -169,8 +169,12 @@ kvc_status kvc_compress_window(kvc_dtype dt, int n_seqs, const int32_t *seqlens_
                                kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Budgeted per-KV-head top-k (SnapKV keeps a chosen subset; the recent window
- * is always kept, as a sliding window keeps its recent region).
+ * Budgeted per-KV-head top-k.  Source: "Variantes de l'attention et
+ * compression du cache KV", section "Compresser un cache existant" (SnapKV
+ * keeps a chosen subset of past keys and values; windowed attention keeps a
+ * bounded recent region, here the w window tokens), and section "Quand la
+ * reutilisation est-elle exacte ?" (positions keep their original indices
+ * after eviction, never renumbered).
  *
  * For sequence b and KV head h: if budget >= len_b the segment is 0..len_b-1.
  * Otherwise it holds the budget - w prefix positions with the largest
@@ -187,9 +191,13 @@ kvc_status kvc_select_topk(int n_seqs, const int32_t *seqlens_host, const int32_
                            const float *scores, int32_t *idx, kvc_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Compact cache gather: for each sequence b, KV head h and slot t <
- * min(budget, len_b):  K_c[cb_b + t][h][:] = K[t0_b + idx[h][cb_b + t]][h][:]
- * and likewise for V (bytes copied unchanged).
+ * Compact cache gather.  Source: "Variantes de l'attention et compression du
+ * cache KV", section "Compresser un cache existant" (the retained keys and
+ * values form the compressed cache); NHD layout of GPU caches from the FreeKV
+ * page, technical summary section 2.B.  For each sequence b, KV head h and
+ * slot t < min(budget, len_b):
+ *   K_c[cb_b + t][h][:] = K[t0_b + idx[h][cb_b + t]][h][:]
+ * and likewise for V (bytes copied unchanged, so the copy is exact).
  *
  * k, v: [T, n_kv, d_h];  k_out, v_out: [cu_budget[n_seqs], n_kv, d_h];  idx
  * as written by kvc_select_topk (every entry must lie in [0, len_b)).

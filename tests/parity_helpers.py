@@ -13,6 +13,17 @@ DECODE_ATOL = {"f32": 1e-5, "bf16": 2e-3}
 TIE_BAND = 1e-5            # selected sets may differ only within this relative band of the k-th score
 
 
+def log_parity(rec):
+    """Append one parity record (JSON line) to $KVC_PARITY_LOG when it is set,
+    so a GPU run can keep the tie-band counts and error maxima of every case."""
+    import json
+    import os
+    path = os.environ.get("KVC_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
 def assert_scores_close(got, ref, rtol=SCORE_RTOL, what="scores"):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
@@ -68,6 +79,19 @@ def assert_selection_matches(idx_gpu, idx_ora, pooled_ora, lengths, w, budget, b
     return n_diff
 
 
+def assert_gather_exact(comp, bt, idx_g, budget):
+    """K_c / V_c against the oracle's byte copy of the rows named by the GPU's
+    index lists (gather is exact given the indices), on every row."""
+    kc_o, vc_o = O.gather_kv(bt["k"], bt["v"], idx_g.astype(np.int64), bt["cu_seqlens"], budget)
+    kc_g, vc_g = from_device(comp.buf.k_c), from_device(comp.buf.v_c)
+    assert kc_g.shape == kc_o.shape and vc_g.shape == vc_o.shape
+    for name, g, o in (("K", kc_g, kc_o), ("V", vc_g, vc_o)):
+        if not np.array_equal(g.view(np.uint8), o.view(np.uint8)):
+            bad = np.argwhere(np.any(g.reshape(g.shape[0], g.shape[1], -1) != o.reshape(o.shape[0], o.shape[1], -1),
+                                     axis=2))
+            raise AssertionError(f"gathered {name} differs on {len(bad)} (slot, head) rows, first {bad[:4].tolist()}")
+
+
 def upload_batch(bt, dtype):
     return to_device(bt["q_win"], dtype), to_device(bt["k"], dtype), to_device(bt["v"], dtype)
 
@@ -101,13 +125,16 @@ def run_and_check_compress(dtype, lengths, n_h, n_kv, d, w, pool_k, budget, seed
     idx_g = comp.buf.idx.cpu().numpy()
     n_diff = assert_selection_matches(idx_g, idx_o, pooled_o, lengths, w, budget)
     if check_gather:
-        kc_o, vc_o = O.gather_kv(bt["k"], bt["v"], idx_o, cu, budget)
-        kc_g, vc_g = from_device(comp.buf.k_c), from_device(comp.buf.v_c)
-        same = (idx_g == idx_o)                       # rows where both sides picked the same token
-        for h in range(n_kv):
-            rows = np.where(same[h])[0]
-            assert np.array_equal(kc_g[rows, h], kc_o[rows, h]), "gathered K differs"
-            assert np.array_equal(vc_g[rows, h], vc_o[rows, h]), "gathered V differs"
+        # the compact caches are bit-exact copies of the rows the GPU's own index
+        # lists name: every row of every head and sequence is compared
+        assert_gather_exact(comp, bt, idx_g, budget)
+    n_rows = int(np.sum(np.minimum(np.asarray(lengths), budget))) * n_kv
+    log_parity(dict(what="compress", dtype=dtype, n_seqs=len(lengths), T=int(np.sum(lengths)), budget=budget,
+                    fused_call=fused_call, tie_band_index_differences=n_diff, retained_rows=n_rows,
+                    gathered_rows_compared=n_rows if check_gather else 0,
+                    max_rel_raw=max_rel(raw_g, raw_o), max_rel_pooled=max_rel(pooled_g, pooled_o)))
+    # the tie band admits a few swaps among equal-looking scores, never a large share
+    assert n_diff <= max(8, n_rows // 100), f"{n_diff} index differences in {n_rows} rows"
     return dict(bt=bt, comp=comp, raw_o=raw_o, pooled_o=pooled_o, idx_o=idx_o, idx_g=idx_g, n_diff=n_diff,
                 dev=(q, k, v))
 
@@ -125,6 +152,8 @@ def run_and_check_decode(dtype, q_np, kc_np, vc_np, offsets, lens, n_kv, max_len
     ref = O.gqa_decode(q_np, kc_np, vc_np, offsets, lens, n_kv, dtype)
     got = out.cpu().numpy().astype(np.float64)
     err = np.abs(got - ref).max()
+    log_parity(dict(what="decode", dtype=dtype, batch=int(batch), n_h=int(n_h), d_h=int(d),
+                    rows=int(np.sum(lens)), max_abs_err=float(err), atol=DECODE_ATOL[dtype]))
     assert err <= DECODE_ATOL[dtype], f"decode max abs error {err:.3e} > {DECODE_ATOL[dtype]}"
     # the completion counters are left at zero for the next call
     tick = dec.ws[256:256 + 4 * batch * n_kv].view(torch.int32)

@@ -18,7 +18,7 @@ import torch
 from kv_cache_compression_score_b200 import synth
 from kv_cache_compression_score_b200.runner import TspSelector, from_device, to_device
 from oracle import kvc_oracle as O
-from parity_helpers import run_and_check_compress, run_and_check_decode
+from parity_helpers import log_parity, run_and_check_compress, run_and_check_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -81,8 +81,9 @@ def test_fastkv_tsp_layer_and_next_layer():
     kth = np.sort(pooled_o)[::-1][k_tsp - 1]
     diff = set(g[:k_tsp].tolist()) ^ set(idx_o[:k_tsp].tolist())
     assert all(abs(pooled_o[j] - kth) <= 1e-5 * kth for j in diff)
-    same = np.where(g == idx_o)[0]
-    assert np.array_equal(from_device(hout)[same], hidden[idx_o[same]])
+    # hidden rows: a byte copy of the rows the GPU's own index list names, every row
+    assert np.array_equal(from_device(hout), O.tsp_gather(hidden, g))
+    log_parity(dict(what="tsp", S=S, k_tsp=k_tsp, tie_band_index_differences=len(diff), rows_compared=len(g)))
     # first layer after the TSP layer runs on S' = k_tsp + w tokens, same KV budget
     run_and_check_compress("bf16", [k_tsp + W], N_H, N_KV, D, W, POOL, kv_budget, seed=1004 + 16, boost_frac=0.01)
 

@@ -28,6 +28,9 @@ def test_small_fp32_layer_s2048_whole_path():
     """One layer, n_h 4, n_kv 2, d_h 64, S 2048, fp32, w 32, pool 7, B 256."""
     r = run_and_check_compress("f32", [2048], 4, 2, 64, 32, 7, 256, seed=1001)
     assert r["n_diff"] == 0
+    # then one decode query over the retained cache (256 rows per KV head)
+    q = synth.decode_queries(1001 + 8, 1, 4, 64, "f32")
+    run_and_check_decode("f32", q, from_device(r["comp"].buf.k_c), from_device(r["comp"].buf.v_c), [0], [256], 2)
 
 
 @pytest.mark.parametrize("lengths", [[1000, 300, 129, 32, 777], [4097]])
@@ -269,5 +272,4 @@ def test_tsp_after_scoring_tie_band():
     diff = set(g[:k_tsp].tolist()) ^ set(idx_o[:k_tsp].tolist())
     kth = np.sort(pooled_o)[::-1][k_tsp - 1]
     assert all(abs(pooled_o[j] - kth) <= 1e-5 * kth for j in diff)
-    same = np.where(g == idx_o)[0]
-    assert np.array_equal(from_device(hout)[same], hidden[idx_o[same]])
+    assert np.array_equal(from_device(hout), O.tsp_gather(hidden, g))

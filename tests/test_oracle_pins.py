@@ -33,6 +33,56 @@ def test_cache_bytes_worked_example():
 
 
 # ---------------------------------------------------------------------------
+# stored inputs: exact widening of bf16 bit patterns
+# ---------------------------------------------------------------------------
+# bf16 is the top half of an IEEE binary32: sign, 8 exponent bits, 7 mantissa
+# bits.  Each pattern below is decoded by hand from that definition.
+BF16_CASES = [
+    (0x3F80, 1.0),                      # exponent 127, mantissa 0
+    (0xC000, -2.0),                     # sign, exponent 128
+    (0xC040, -3.0),                     # exponent 128, mantissa 0b1000000 -> 1.5 * 2
+    (0x4049, 3.140625),                 # exponent 128, mantissa 0b1001001 -> (1 + 73/128) * 2
+    (0x3E80, 0.25),                     # exponent 125
+    (0x0001, 2.0 ** -133),              # smallest subnormal: 2^-126 * 2^-7
+    (0x007F, 127 * 2.0 ** -133),        # largest subnormal
+    (0x0080, 2.0 ** -126),              # smallest normal
+    (0x7F7F, (2 - 2.0 ** -7) * 2.0 ** 127),   # largest finite
+    (0x8000, -0.0),
+    (0x0000, 0.0),
+    (0x7F80, math.inf),
+    (0xFF80, -math.inf),
+]
+
+
+def test_bf16_widening_hand_decoded_patterns():
+    bits = np.array([b for b, _ in BF16_CASES], dtype=np.uint16)
+    got = O.to_f64(bits, "bf16")
+    for (b, want), g in zip(BF16_CASES, got):
+        assert g == want and math.copysign(1.0, g) == math.copysign(1.0, want), f"0x{b:04X}: {g!r} != {want!r}"
+    nan = O.to_f64(np.array([0x7FC0, 0xFFC1], dtype=np.uint16), "bf16")
+    assert np.all(np.isnan(nan))
+
+
+def test_bf16_widening_matches_torch_on_every_pattern():
+    """All 65536 patterns against torch's own bf16 -> float64 conversion of
+    the same bits (an implementation that shares nothing with the oracle)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = O.to_f64(bits, "bf16")
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    fin = ~np.isnan(ref)
+    assert np.array_equal(np.isnan(got), ~fin)
+    assert np.array_equal(got[fin], ref[fin])
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(ref[fin]))
+
+
+def test_f32_widening_is_the_identity_on_values():
+    x = np.array([1.0, -2.5, 2.0 ** -149, 3.4028234663852886e38, -0.0], dtype=np.float32)
+    got = O.to_f64(x, "f32")
+    assert np.array_equal(got, np.array([1.0, -2.5, 2.0 ** -149, 3.4028234663852886e38, -0.0]))
+    assert math.copysign(1.0, got[4]) == -1.0
+
+
+# ---------------------------------------------------------------------------
 # scoring: closed forms
 # ---------------------------------------------------------------------------
 def _batch(lengths, n_h, n_kv, d, w, seed=7, dtype="f32"):

@@ -48,6 +48,27 @@ def test_static_scratch_matches_workspace_variant_twice():
         assert np.array_equal(from_device(hid), from_device(hid_ref))
 
 
+def test_static_scratch_at_its_limit():
+    """S - w exactly at the array's capacity (262,144 pooled prefix scores):
+    the last element of the array is written and read; one more is refused."""
+    w, pool_k, k_tsp, D = 32, 7, 300, 8
+    S = 262144 + w
+    raw, hidden = _case(93, S, w, 1, k_tsp, D)
+    ref = TspSelector(S, w, pool_k, k_tsp, D, "bf16")
+    idx_ref, hid_ref = ref.run(raw, hidden)
+    idx = torch.empty(k_tsp + w, dtype=torch.int32, device="cuda")
+    hid = torch.empty((k_tsp + w, D), dtype=torch.bfloat16, device="cuda")
+    kvc.kvc_tsp_select_gather_static(raw, w, pool_k, k_tsp, hidden, idx, hid)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_ref.cpu().numpy())
+    assert np.array_equal(from_device(hid), from_device(hid_ref))
+    raw1 = torch.zeros((1, S + 1), dtype=torch.float32, device="cuda")
+    hidden1 = torch.zeros((S + 1, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_tsp_select_gather_static(raw1, w, pool_k, k_tsp, hidden1, idx, hid)
+    assert e.value.status == kvc.KVC_ERR_UNSUPPORTED
+
+
 def test_static_scratch_rejects_oversize():
     S, w = 262144 + 64, 32
     raw = torch.zeros((1, S), dtype=torch.float32, device="cuda")
