@@ -32,6 +32,11 @@ or bf16 bit patterns, both widened exactly):
    of k_tsp prefix positions plus the window, hidden rows copied.
 8. ``cache_bytes`` -- 2 * L * S * n_kv * d_h * b (attention-variants page,
    section "MHA et GQA").
+9. ``quantize_rows_int8`` / ``gather_kv_q8`` / ``gqa_decode_q8`` -- the KV cache
+   stored at lower precision (attention-variants page, section "Compresser un
+   cache existant": cache quantisation): every retained (row, head) vector is
+   stored as int8 codes with one float32 scale, and decode attention runs over
+   the dequantised values.
 
 Every function above is pinned by tests/test_oracle_pins.py (closed forms,
 invariants, the pages' worked cache-size example, brute force on tiny inputs,
@@ -47,7 +52,11 @@ Readings of points the pages leave open:
 * pool: stride 1, same length, neighbours outside [0, P) ignored;
 * the per-head budget B counts the window (B - w prefix positions);
   the TSP count k_tsp does not (k_tsp + w rows);
-* B >= len keeps every position; B < w is rejected; even pool sizes rejected.
+* B >= len keeps every position; B < w is rejected; even pool sizes rejected;
+* quantised cache: symmetric int8 per (row, head) vector, scale = max|x| / 127
+  and code = round-half-even(x / scale), both quotients in float32 (the
+  precision the stored values have), codes clipped to [-127, 127]; an all-zero
+  vector has scale 0 and codes 0.  Dequantised value = code * scale.
 
 Parity pins for every function live in tests/test_oracle_pins.py; none of them
 re-types these formulas.
@@ -67,6 +76,8 @@ def to_f64(x: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "bf16":
         bits = np.asarray(x, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
         return bits.view(np.float32).astype(np.float64)
+    if dtype == "f64":
+        return np.asarray(x, dtype=np.float64)
     raise ValueError(f"unknown dtype {dtype!r}")
 
 
@@ -257,12 +268,15 @@ def gather_kv(k: np.ndarray, v: np.ndarray, idx: np.ndarray, cu_seqlens, budget:
 # 6. decode attention
 # ----------------------------------------------------------------------------
 def gqa_decode(q: np.ndarray, k_c: np.ndarray, v_c: np.ndarray, row_offset, kv_len,
-               n_kv: int, dtype: str, scale: float | None = None) -> np.ndarray:
+               n_kv: int, dtype: str, scale: float | None = None, cache_dtype: str | None = None) -> np.ndarray:
     """out[b, qh] = sum_t softmax_t(scale * q[b, qh] . K_c[off_b + t, qh // G]) V_c[off_b + t, qh // G]
-    over t < kv_len[b]; an empty cache gives 0.  float64 [batch, n_h, d]."""
+    over t < kv_len[b]; an empty cache gives 0.  float64 [batch, n_h, d].
+    cache_dtype (default: dtype) names the stored type of k_c / v_c; "f64"
+    takes them as float64 values."""
+    cache_dtype = dtype if cache_dtype is None else cache_dtype
     qf = to_f64(q, dtype)
-    kf = to_f64(k_c, dtype)
-    vf = to_f64(v_c, dtype)
+    kf = to_f64(k_c, cache_dtype)
+    vf = to_f64(v_c, cache_dtype)
     batch, n_h, d = qf.shape
     if scale is None or scale <= 0:
         scale = default_scale(d)
@@ -310,3 +324,47 @@ def tsp_gather(hidden: np.ndarray, idx: np.ndarray) -> np.ndarray:
 def rate_count(rate: float, S: int) -> int:
     """Token count of a rate applied to S tokens (reading: floor)."""
     return int(np.floor(rate * S))
+
+
+# ----------------------------------------------------------------------------
+# 9. quantised compact cache
+# ----------------------------------------------------------------------------
+def quantize_rows_int8(x: np.ndarray):
+    """Symmetric int8 quantisation of every vector along the last axis.
+
+    x: float32 values (the exact widening of the stored cache).  Returns
+    (codes int8 of x's shape, scales float32 of x.shape[:-1]).  The scale is
+    max|x| / 127 and the code round-half-even(x / scale), each quotient taken
+    in float32; all-zero vectors get scale 0 and codes 0."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    ratio = (x / safe[..., None]).astype(np.float32)
+    codes = np.clip(np.rint(ratio), -127, 127)
+    codes = np.where(scale[..., None] > 0, codes, 0).astype(np.int8)
+    return codes, scale
+
+
+def dequantize_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """code * scale in float64 (exact: an 8-bit integer times a float32)."""
+    return codes.astype(np.float64) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+def gather_kv_q8(k: np.ndarray, v: np.ndarray, idx: np.ndarray, cu_seqlens, budget: int, dtype: str):
+    """Gather the retained rows (as gather_kv) and quantise every (slot, head)
+    vector.  Returns (kq, vq int8 [Tb, n_kv, d], ks, vs float32 [n_kv, Tb])."""
+    kc, vc = gather_kv(k, v, idx, cu_seqlens, budget)
+    kq, ks = quantize_rows_int8(to_f64(kc, dtype).astype(np.float32))
+    vq, vs = quantize_rows_int8(to_f64(vc, dtype).astype(np.float32))
+    return kq, vq, np.ascontiguousarray(ks.T), np.ascontiguousarray(vs.T)
+
+
+def gqa_decode_q8(q: np.ndarray, kq: np.ndarray, vq: np.ndarray, k_scale: np.ndarray, v_scale: np.ndarray,
+                  row_offset, kv_len, n_kv: int, q_dtype: str, scale: float | None = None) -> np.ndarray:
+    """Decode attention (gqa_decode) over the dequantised int8 caches.
+    k_scale, v_scale: [n_kv, >= rows] float32."""
+    rows = kq.shape[0]
+    kd = dequantize_rows(kq, np.asarray(k_scale)[:, :rows].T)
+    vd = dequantize_rows(vq, np.asarray(v_scale)[:, :rows].T)
+    return gqa_decode(q, kd, vd, row_offset, kv_len, n_kv, q_dtype, scale, cache_dtype="f64")

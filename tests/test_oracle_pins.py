@@ -408,3 +408,83 @@ def test_generators_deterministic_and_normal():
     assert lens.min() >= 4096 and lens.max() <= 65536
     pos = synth.boosted_positions(1002, 0, 0, 32768, 0.01)
     assert len(pos) == 327 and len(np.unique(pos)) == 327
+
+
+# ---------------------------------------------------------------------------
+# quantised compact cache (int8 codes, one float32 scale per (row, head))
+# ---------------------------------------------------------------------------
+def test_quantize_exact_power_of_two_rows():
+    """max|x| = 127 * 2^e and every element a multiple of 2^e: the scale is
+    exactly 2^e, the codes are x / 2^e and dequantisation gives x back."""
+    for e in (-7, 0, 3):
+        codes = np.array([[127, -5, 0, 64, -127, 1], [-127, 2, 3, -4, 100, 7]], dtype=np.int64)
+        x = (codes * 2.0 ** e).astype(np.float32)
+        q, s = O.quantize_rows_int8(x)
+        assert q.dtype == np.int8 and s.dtype == np.float32
+        np.testing.assert_array_equal(s, [2.0 ** e, 2.0 ** e])
+        np.testing.assert_array_equal(q, codes)
+        np.testing.assert_array_equal(O.dequantize_rows(q, s), x.astype(np.float64))
+
+
+def test_quantize_rounds_half_to_even_and_clips():
+    """Scale 1 (max|x| = 127): x / scale = x, so the codes are x rounded half
+    to even -- 2.5 -> 2, -2.5 -> -2, 3.5 -> 4, 0.5 -> 0, -0.5 -> -0."""
+    x = np.array([[127.0, 2.5, -2.5, 3.5, 0.5, -0.5, 126.49, -126.51]], dtype=np.float32)
+    q, s = O.quantize_rows_int8(x)
+    assert s[0] == 1.0
+    np.testing.assert_array_equal(q[0], [127, 2, -2, 4, 0, 0, 126, -127])
+
+
+def test_quantize_zero_row_and_error_bound():
+    x = synth.normal_tensor(77, synth.T_K, 0, (64, 128), "f32")
+    x[5] = 0.0
+    q, s = O.quantize_rows_int8(x)
+    assert s[5] == 0.0 and np.all(q[5] == 0)
+    assert np.all(np.abs(q.astype(np.int64)) <= 127)
+    for r in range(64):
+        if r == 5:
+            continue
+        j = np.argmax(np.abs(x[r]))
+        assert abs(int(q[r, j])) == 127                      # the largest element maps to +-127
+        err = np.abs(x[r].astype(np.float64) - O.dequantize_rows(q[r:r + 1], s[r:r + 1])[0])
+        assert err.max() <= 0.5 * float(s[r]) * (1 + 2.0 ** -20)   # half a quantisation step
+    # scaling a row by a power of two scales the scale and keeps the codes
+    q2, s2 = O.quantize_rows_int8((x * np.float32(8.0)).astype(np.float32))
+    np.testing.assert_array_equal(q2, q)
+    np.testing.assert_array_equal(s2, s * np.float32(8.0))
+
+
+def test_gather_q8_is_gather_then_quantize_per_head_row():
+    lengths, n_kv, d, w, B = [40, 9], 2, 16, 4, 12
+    bt = synth.packed_batch(81, lengths, 4, n_kv, d, w, "bf16")
+    idx = synth.index_lists(82, lengths, n_kv, B).astype(np.int64)
+    kq, vq, ks, vs = O.gather_kv_q8(bt["k"], bt["v"], idx, bt["cu_seqlens"], B, "bf16")
+    kc, vc = O.gather_kv(bt["k"], bt["v"], idx, bt["cu_seqlens"], B)
+    assert kq.shape == kc.shape and ks.shape == (n_kv, kc.shape[0])
+    for t in range(kc.shape[0]):
+        for h in range(n_kv):
+            row = O.to_f64(kc[t, h], "bf16").astype(np.float32)
+            amax = np.max(np.abs(row))
+            assert ks[h, t] == np.float32(amax) / np.float32(127)
+            np.testing.assert_array_equal(kq[t, h], np.clip(np.rint(row / ks[h, t]), -127, 127))
+
+
+def test_decode_q8_lossless_cache_equals_plain_decode():
+    """A cache whose rows hold integers in [-127, 127] with +-127 present is
+    quantised without loss (scale 1), so decode over it equals decode over
+    the plain float32 cache; scaling the cache by 2^-4 scales only the
+    scales."""
+    n_h, n_kv, d, rows = 8, 2, 16, 50
+    u = synth.uniform_u64(synth.stream_key(91, synth.T_K, 0), rows * n_kv * d)
+    ints = ((u % np.uint64(255)).astype(np.int64) - 127).reshape(rows, n_kv, d)
+    ints[:, :, 0] = 127
+    kf = (ints * 2.0 ** -4).astype(np.float32)
+    vf = (ints[::-1] * 2.0 ** -4).astype(np.float32)
+    kq, ks = O.quantize_rows_int8(kf)
+    vq, vs = O.quantize_rows_int8(vf)
+    assert np.all(ks == 2.0 ** -4) and np.all(vs == 2.0 ** -4)
+    q = synth.decode_queries(92, 3, n_h, d, "bf16")
+    offs, lens = [0, 10, 0], [50, 40, 1]
+    got = O.gqa_decode_q8(q, kq, vq, ks.T, vs.T, offs, lens, n_kv, "bf16")
+    ref = O.gqa_decode(q, kf, vf, offs, lens, n_kv, "bf16", cache_dtype="f32")
+    np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
