@@ -115,6 +115,20 @@ uint64_t kvc_cache_bytes(int L, int64_t S, int n_kv, int d_h, int b);
 int64_t kvc_budget_offsets(int n_seqs, const int32_t *seqlens_host, int budget,
                            int32_t *cu_budget_host);
 
+/*
+ * PyramidKV per-layer budgets (host only).  Source: "Variantes de l'attention
+ * et compression du cache KV", section "Compresser un cache existant":
+ * PyramidKV gives different layers different cache budgets.  The page gives no
+ * shape; this library's reading is the arithmetic sequence falling from
+ * B_max = 2 * avg_budget - min_budget at layer 0 to min_budget at layer L - 1:
+ *   budgets_host[l] = B_max - floor((B_max - min_budget) * l / (L - 1))
+ * (L == 1: avg_budget), so the mean is avg_budget, rounded up by less than one
+ * token per layer.  Each layer then calls kvc_compress_window with its own
+ * budget.  Returns the sum of the budgets, or -1 on invalid input (L < 1,
+ * min_budget < 0, min_budget > avg_budget, NULL output).
+ */
+int64_t kvc_pyramid_budgets(int L, int avg_budget, int min_budget, int32_t *budgets_host);
+
 /* ------------------------------------------------------------------------
  * Window saliency scores (SnapKV observation window; FastKV 2.A saliency).
  *
@@ -269,6 +283,38 @@ kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d
                                const int64_t *kv_row_offset, const int32_t *kv_len,
                                int max_kv_len, float *out, void *ws, size_t ws_bytes,
                                kvc_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Quantised compact cache.  Source: "Variantes de l'attention et compression
+ * du cache KV", section "Compresser un cache existant" (KV-cache quantisation
+ * stores the cache elements at a lower precision; custom layouts need their
+ * own kernels).  Format: int8 codes in the compact cache's NHD layout
+ * [rows, n_kv, d_h] plus one float32 scale per (row, head) in
+ * [n_kv, scale_pitch]; the value a code stands for is code * scale.
+ *
+ * kvc_gather_kv_q8: the gather of kvc_gather_kv from bf16 caches k, v, and
+ * for every retained (slot, head) vector x: scale = max|x| / 127 and code =
+ * round-half-even(x / scale) clipped to [-127, 127], both quotients IEEE
+ * float32 divisions (a zero vector: scale 0, codes 0).  k_q, v_q: int8
+ * [cu_budget[n_seqs], n_kv, d_h]; k_scale, v_scale: float32 [n_kv,
+ * scale_pitch], scale_pitch >= cu_budget[n_seqs].  d_h in {64, 128}.
+ * ------------------------------------------------------------------------ */
+kvc_status kvc_gather_kv_q8(int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                            const int32_t *cu_budget, int n_kv, int d_h, int budget, const int32_t *idx,
+                            const void *k, const void *v, int8_t *k_q, int8_t *v_q, float *k_scale,
+                            float *v_scale, int64_t scale_pitch, kvc_stream_t stream);
+
+/* kvc_gqa_decode_attn_q8: kvc_gqa_decode_attn over int8 caches, with the
+ * logits and weights of the dequantised values code * scale (the K scale of
+ * a row multiplies its logit, the V scale its weight).  q: bf16 [batch, n_h,
+ * d_h]; k_q, v_q: int8 [cache_rows, n_kv, d_h]; k_scale, v_scale: float32
+ * [n_kv, scale_pitch], scale_pitch >= cache_rows.  Other arguments, the
+ * workspace (kvc_gqa_decode_workspace_size) and errors as kvc_gqa_decode_attn. */
+kvc_status kvc_gqa_decode_attn_q8(int batch, int n_h, int n_kv, int d_h, float scale, const void *q,
+                                  const int8_t *k_q, const int8_t *v_q, const float *k_scale,
+                                  const float *v_scale, int64_t scale_pitch, int64_t cache_rows,
+                                  const int64_t *kv_row_offset, const int32_t *kv_len, int max_kv_len,
+                                  float *out, void *ws, size_t ws_bytes, kvc_stream_t stream);
 
 #ifdef __cplusplus
 }

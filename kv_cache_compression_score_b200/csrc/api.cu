@@ -216,6 +216,22 @@ int64_t kvc_budget_offsets(int n_seqs, const int32_t *seqlens_host, int budget, 
   return acc;
 }
 
+int64_t kvc_pyramid_budgets(int L, int avg_budget, int min_budget, int32_t *budgets_host) {
+  if (L < 1 || min_budget < 0 || min_budget > avg_budget || !budgets_host) return -1;
+  if (L == 1) {
+    budgets_host[0] = avg_budget;
+    return avg_budget;
+  }
+  const int64_t b_max = 2 * (int64_t)avg_budget - min_budget;
+  if (b_max > INT32_MAX) return -1;
+  int64_t total = 0;
+  for (int l = 0; l < L; ++l) {
+    budgets_host[l] = (int32_t)(b_max - ((b_max - min_budget) * l) / (L - 1));
+    total += budgets_host[l];
+  }
+  return total;
+}
+
 size_t kvc_score_window_workspace_size(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int n_h, int n_kv,
                                        int d_h, int w) {
   ScorePlan pl;
@@ -379,6 +395,36 @@ kvc_status kvc_gather_kv(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, 
   return KVC_OK;
 }
 
+kvc_status kvc_gather_kv_q8(int n_seqs, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                            const int32_t *cu_budget, int n_kv, int d_h, int budget, const int32_t *idx, const void *k,
+                            const void *v, int8_t *k_q, int8_t *v_q, float *k_scale, float *v_scale,
+                            int64_t scale_pitch, kvc_stream_t stream) {
+  Batch bt;
+  kvc_status s = check_batch(n_seqs, seqlens_host, 0, &bt);
+  if (s != KVC_OK) return s;
+  if (n_kv < 1) return fail(KVC_ERR_INVALID_ARG, "n_kv must be >= 1");
+  if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
+  if (budget < 0) return fail(KVC_ERR_INVALID_ARG, "budget must be >= 0");
+  if (!cu_seqlens || !cu_budget) return fail(KVC_ERR_INVALID_ARG, "cu_seqlens / cu_budget is NULL");
+  if (!aligned16(idx) || !aligned16(k) || !aligned16(v) || !aligned16(k_q) || !aligned16(v_q) ||
+      !aligned16(k_scale) || !aligned16(v_scale))
+    return fail(KVC_ERR_INVALID_ARG, "idx, k, v, k_q, v_q, k_scale and v_scale must be non-NULL and 16-byte aligned");
+  int64_t total = 0;
+  int max_kept = 0;
+  for (int b = 0; b < n_seqs; ++b) {
+    const int kept = std::min(budget, seqlens_host[b]);
+    total += kept;
+    max_kept = std::max(max_kept, kept);
+  }
+  if (scale_pitch < total) return fail(KVC_ERR_INVALID_ARG, "scale_pitch (%lld) must be >= the %lld compact rows",
+                                       (long long)scale_pitch, (long long)total);
+  if (total == 0) return KVC_OK;
+  cudaError_t e = kvc::gather_rows_kv_q8(k, v, k_q, v_q, k_scale, v_scale, scale_pitch, idx, cu_seqlens, cu_budget,
+                                         n_seqs, n_kv, d_h, (int)total, max_kept, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather-and-quantise kernel");
+  return KVC_OK;
+}
+
 size_t kvc_tsp_workspace_size(int S, int w) {
   if (S < 1 || w < 1 || w > S) return 0;
   return kErrWordBytes + round_up((size_t)(S - w) * sizeof(float), 256);
@@ -445,6 +491,42 @@ kvc_status kvc_gqa_decode_attn(kvc_dtype dt, int batch, int n_h, int n_kv, int d
   a.chunk_rows = pl.chunk_rows;
   cudaError_t e = kvc::gqa_decode(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
+  return KVC_OK;
+}
+
+kvc_status kvc_gqa_decode_attn_q8(int batch, int n_h, int n_kv, int d_h, float scale, const void *q,
+                                  const int8_t *k_q, const int8_t *v_q, const float *k_scale, const float *v_scale,
+                                  int64_t scale_pitch, int64_t cache_rows, const int64_t *kv_row_offset,
+                                  const int32_t *kv_len, int max_kv_len, float *out, void *ws, size_t ws_bytes,
+                                  kvc_stream_t stream) {
+  DecodePlan pl;
+  kvc_status s = plan_decode(KVC_BF16, batch, n_h, n_kv, d_h, max_kv_len, &pl);
+  if (s != KVC_OK) return s;
+  if (!aligned16(q) || !aligned16(k_q) || !aligned16(v_q) || !aligned16(out) || !aligned16(k_scale) ||
+      !aligned16(v_scale))
+    return fail(KVC_ERR_INVALID_ARG, "q, k_q, v_q, k_scale, v_scale and out must be non-NULL and 16-byte aligned");
+  if (!kv_row_offset || !kv_len) return fail(KVC_ERR_INVALID_ARG, "kv_row_offset / kv_len is NULL");
+  if (cache_rows < 1 || cache_rows > INT32_MAX)
+    return fail(KVC_ERR_INVALID_ARG, "cache_rows must lie in [1, 2^31) (got %lld)", (long long)cache_rows);
+  if (scale_pitch < cache_rows)
+    return fail(KVC_ERR_INVALID_ARG, "scale_pitch (%lld) must be >= cache_rows (%lld)", (long long)scale_pitch,
+                (long long)cache_rows);
+  if (!aligned16(ws) || ws_bytes < pl.bytes)
+    return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", pl.bytes, ws_bytes);
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_h);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  kvc::DecodeArgs a;
+  a.dt = KVC_BF16; a.batch = batch; a.n_h = n_h; a.n_kv = n_kv; a.d_h = d_h; a.scale = scale;
+  a.q = q; a.k_c = k_q; a.v_c = v_q; a.row_off = kv_row_offset; a.kv_len = kv_len; a.out = out;
+  a.tickets = reinterpret_cast<int *>(wsb + pl.off_tickets);
+  a.err = reinterpret_cast<int *>(wsb);
+  a.cache_rows = cache_rows;
+  a.part = reinterpret_cast<float *>(wsb + pl.off_part);
+  a.n_chunks = pl.n_chunks;
+  a.chunk_rows = pl.chunk_rows;
+  a.k_scale = k_scale; a.v_scale = v_scale; a.scale_pitch = scale_pitch;
+  cudaError_t e = kvc::gqa_decode_tc(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "int8 decode kernel");
   return KVC_OK;
 }
 

@@ -1,4 +1,4 @@
-// GQA decode attention over compact caches: out[b, qh] = softmax(scale *
+// GQA decode attention over float32 compact caches: out[b, qh] = softmax(scale *
 // q[b, qh] . Kc[o_b + t, h]) . Vc[o_b + t, h], h = qh / G.  Decode streams
 // the whole retained cache every step, so the kernel is an HBM stream (FastKV
 // section 1; "Variantes de l'attention et compression du cache KV",
@@ -433,9 +433,11 @@ cudaError_t by_group(const DecodeArgs &a, cudaStream_t st) {
 // len / kMinRowsPerWarp + 2 slices.
 int decode_slots(int max_kv_len) { return max_kv_len / kMinRowsPerWarp + 2; }
 
+// float32 caches run on the CUDA cores (full fp32 products); bf16 and int8
+// caches go to the tensor-core kernel (decode_mma.cu)
 cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st) {
   if (a.dt == KVC_F32) return a.d_h == 64 ? by_group<float, 64>(a, st) : by_group<float, 128>(a, st);
-  return a.d_h == 64 ? by_group<__nv_bfloat16, 64>(a, st) : by_group<__nv_bfloat16, 128>(a, st);
+  return gqa_decode_tc(a, st);
 }
 
 }  // namespace kvc

@@ -58,6 +58,11 @@ cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_ou
                            const int32_t *cu_seqlens, const int32_t *cu_budget, int n_seqs, int n_kv,
                            int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st);
 
+cudaError_t gather_rows_kv_q8(const void *k, const void *v, int8_t *kq, int8_t *vq, float *ks, float *vs,
+                              int64_t scale_pitch, const int32_t *idx, const int32_t *cu_seqlens,
+                              const int32_t *cu_budget, int n_seqs, int n_kv, int d_h, int total_budget, int max_kept,
+                              cudaStream_t st);
+
 cudaError_t tsp_pool(const float *raw, int n_rows, int S, int w, int pool_k, float *pooled, cudaStream_t st);
 cudaError_t tsp_select(const float *pooled, int S, int w, int k_tsp, int32_t *idx_out, cudaStream_t st);
 cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int n_rows, int row_bytes, int n_src,
@@ -77,8 +82,12 @@ struct DecodeArgs {
   int64_t cache_rows;    // rows of k_c / v_c
   int n_chunks;          // partial slots per (batch entry, KV head)
   int chunk_rows;        // unused by the stream-K kernel (kept 0)
+  // int8 caches (k_c / v_c hold int8 codes): per-(row, head) scales [n_kv, scale_pitch]
+  const float *k_scale = nullptr, *v_scale = nullptr;
+  int64_t scale_pitch = 0;
 };
 cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
+cudaError_t gqa_decode_tc(const DecodeArgs &a, cudaStream_t st);   // bf16 / int8 caches, tensor cores
 int decode_slots(int max_kv_len);
 
 }  // namespace kvc

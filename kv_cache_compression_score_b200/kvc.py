@@ -31,6 +31,7 @@ SIGNATURES = {
     "kvc_last_error": (ctypes.c_char_p, []),
     "kvc_cache_bytes": (_c_u64, [_c_int, _c_i64, _c_int, _c_int, _c_int]),
     "kvc_budget_offsets": (_c_i64, [_c_int, _c_p, _c_int, _c_p]),
+    "kvc_pyramid_budgets": (_c_i64, [_c_int, _c_int, _c_int, _c_p]),
     "kvc_score_window_workspace_size": (_c_sz, [_c_int, _c_int, _c_p, _c_int, _c_int, _c_int, _c_int]),
     "kvc_score_window": (_c_int, [_c_int, _c_int, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_f,
                                   _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
@@ -45,6 +46,10 @@ SIGNATURES = {
                                        _c_p, _c_p, _c_sz, _c_p]),
     "kvc_tsp_select_gather_static": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p, _c_int,
                                               _c_p, _c_p, _c_p]),
+    "kvc_gather_kv_q8": (_c_int, [_c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_p, _c_p, _c_p, _c_p, _c_p,
+                                  _c_p, _c_p, _c_i64, _c_p]),
+    "kvc_gqa_decode_attn_q8": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
+                                        _c_i64, _c_p, _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
     "kvc_gqa_decode_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_i64, _c_p,
                                      _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
@@ -140,6 +145,15 @@ def kvc_budget_offsets(seqlens, budget: int) -> np.ndarray:
     return out
 
 
+def kvc_pyramid_budgets(L: int, avg_budget: int, min_budget: int) -> np.ndarray:
+    """Per-layer PyramidKV budgets (host helper of the library)."""
+    out = np.zeros(max(L, 1), dtype=np.int32)
+    total = lib().kvc_pyramid_budgets(L, avg_budget, min_budget, out.ctypes.data_as(ctypes.c_void_p))
+    if total < 0:
+        raise KvcError(1, "kvc_pyramid_budgets: invalid input")
+    return out
+
+
 def kvc_score_window_workspace_size(dt: int, seqlens, n_h: int, n_kv: int, d_h: int, w: int) -> int:
     sl, p = _host_i32(seqlens)
     return int(lib().kvc_score_window_workspace_size(dt, len(sl), p, n_h, n_kv, d_h, w))
@@ -210,3 +224,21 @@ def kvc_gqa_decode_attn(q, k_c, v_c, kv_row_offset, kv_len, max_kv_len: int, sca
                                      _dptr(v_c), k_c.shape[0], _dptr(kv_row_offset), _dptr(kv_len), max_kv_len,
                                      _dptr(out),
                                      _dptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_gather_kv_q8(seqlens, cu_seqlens, cu_budget, budget: int, idx, k, v, k_q, v_q, k_scale, v_scale,
+                     stream=None) -> None:
+    """Gather the retained rows of bf16 caches and quantise each (slot, head) vector to int8 + a float32 scale."""
+    sl, p = _host_i32(seqlens)
+    _check(lib().kvc_gather_kv_q8(len(sl), p, _dptr(cu_seqlens), _dptr(cu_budget), k.shape[1], k.shape[2], budget,
+                                  _dptr(idx), _dptr(k), _dptr(v), _dptr(k_q), _dptr(v_q), _dptr(k_scale),
+                                  _dptr(v_scale), k_scale.shape[1], _stream(stream)))
+
+
+def kvc_gqa_decode_attn_q8(q, k_q, v_q, k_scale, v_scale, kv_row_offset, kv_len, max_kv_len: int, scale: float, out,
+                           ws, stream=None) -> None:
+    batch, n_h, d_h = q.shape
+    _check(lib().kvc_gqa_decode_attn_q8(batch, n_h, k_q.shape[1], d_h, scale, _dptr(q), _dptr(k_q), _dptr(v_q),
+                                        _dptr(k_scale), _dptr(v_scale), k_scale.shape[1], k_q.shape[0],
+                                        _dptr(kv_row_offset), _dptr(kv_len), max_kv_len, _dptr(out), _dptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)))

@@ -37,6 +37,16 @@ or bf16 bit patterns, both widened exactly):
    cache existant": cache quantisation): every retained (row, head) vector is
    stored as int8 codes with one float32 scale, and decode attention runs over
    the dequantised values.
+11. ``freekv_flags`` / ``decode_query_scores`` / ``freekv_step`` -- FreeKV's
+   decode-time retrieval with fine-grained correction (FreeKV, technical
+   summary 2.A): a step reuses the token set retrieved for the previous step;
+   a KV head whose query has drifted -- cosine similarity between the current
+   and the previous query below tau -- is scored again with the current
+   query, its tokens are selected again and retrieved before attention.
+10. ``pyramid_budgets`` -- PyramidKV's per-layer cache budgets (attention-variants
+   page, section "Compresser un cache existant": different layers get different
+   budgets): a budget that falls linearly from the first layer to the last
+   around a given mean.
 
 Every function above is pinned by tests/test_oracle_pins.py (closed forms,
 invariants, the pages' worked cache-size example, brute force on tiny inputs,
@@ -53,6 +63,21 @@ Readings of points the pages leave open:
 * the per-head budget B counts the window (B - w prefix positions);
   the TSP count k_tsp does not (k_tsp + w rows);
 * B >= len keeps every position; B < w is rejected; even pool sizes rejected;
+* PyramidKV schedule (the page gives no shape): for L layers, a mean budget
+  B_avg and a last-layer budget B_min <= B_avg, layer l keeps
+  B_max - floor((B_max - B_min) * l / (L - 1)) tokens per KV head, with
+  B_max = 2 * B_avg - B_min -- the arithmetic sequence from B_max down to B_min
+  whose mean is B_avg, rounded so that the total is never below L * B_avg;
+  a single layer keeps B_avg;
+* FreeKV: the similarity of a KV head is the smallest cosine over the query
+  heads of its group (cosine 0 when a vector is zero); the head is corrected
+  when it is below tau.  A corrected head is scored as in the observation
+  window, with the current decode query as the only window row, seeing every
+  cached key: raw[j] = sum over the group of softmax_j(scale * q . k_j); the
+  same pool over the prefix [0, len - w) and the same budgeted selection (the
+  w most recent tokens always kept) then pick its tokens.  Heads above tau
+  keep their index list (and compact rows); decode attention then runs over
+  every head's compact cache;
 * quantised cache: symmetric int8 per (row, head) vector, scale = max|x| / 127
   and code = round-half-even(x / scale), both quotients in float32 (the
   precision the stored values have), codes clipped to [-127, 127]; an all-zero
@@ -368,3 +393,80 @@ def gqa_decode_q8(q: np.ndarray, kq: np.ndarray, vq: np.ndarray, k_scale: np.nda
     kd = dequantize_rows(kq, np.asarray(k_scale)[:, :rows].T)
     vd = dequantize_rows(vq, np.asarray(v_scale)[:, :rows].T)
     return gqa_decode(q, kd, vd, row_offset, kv_len, n_kv, q_dtype, scale, cache_dtype="f64")
+
+
+# ----------------------------------------------------------------------------
+# 10. PyramidKV per-layer budgets
+# ----------------------------------------------------------------------------
+def pyramid_budgets(L: int, avg_budget: int, min_budget: int) -> np.ndarray:
+    """Per-layer budgets falling linearly from 2 * avg - min (layer 0) to min
+    (layer L - 1), integer arithmetic throughout.  int64 [L]."""
+    if L < 1 or min_budget < 0 or min_budget > avg_budget:
+        raise ValueError("need L >= 1 and 0 <= min_budget <= avg_budget")
+    if L == 1:
+        return np.array([avg_budget], dtype=np.int64)
+    b_max = 2 * avg_budget - min_budget
+    return np.array([b_max - ((b_max - min_budget) * l) // (L - 1) for l in range(L)], dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# 11. FreeKV decode-time retrieval with fine-grained correction
+# ----------------------------------------------------------------------------
+def freekv_flags(q_cur: np.ndarray, q_prev: np.ndarray, n_kv: int, tau: float, dtype: str):
+    """(flags bool [batch, n_kv], cos float64 [batch, n_h]): cos of the current
+    and previous query of every query head; a KV head is flagged (scored and
+    selected again) when the smallest cos of its group is below tau."""
+    a = to_f64(q_cur, dtype)
+    b = to_f64(q_prev, dtype)
+    dot = np.sum(a * b, axis=-1)
+    den = np.sqrt(np.sum(a * a, axis=-1)) * np.sqrt(np.sum(b * b, axis=-1))
+    cos = np.where(den > 0, dot / np.where(den > 0, den, 1.0), 0.0)
+    batch, n_h = cos.shape
+    G = n_h // n_kv
+    return cos.reshape(batch, n_kv, G).min(axis=2) < tau, cos
+
+
+def decode_query_scores(q: np.ndarray, k: np.ndarray, cu_seqlens, n_kv: int, dtype: str,
+                        scale: float | None = None) -> np.ndarray:
+    """raw[h, t]: for sequence b, the softmax mass that the decode queries of
+    the G query heads of KV head h put on each of its len_b cached keys (the
+    query follows the whole cache, so every key is visible).  [n_kv, T]."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    qf = to_f64(q, dtype)
+    kf = to_f64(k, dtype)
+    batch, n_h, d = qf.shape
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    G = n_h // n_kv
+    out = np.zeros((n_kv, int(cu[-1])))
+    for b in range(batch):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        for h in range(n_kv):
+            z = scale * (qf[b, h * G:(h + 1) * G] @ kf[t0:t1, h].T)        # [G, len]
+            e = np.exp(z - z.max(axis=1, keepdims=True))
+            out[h, t0:t1] = (e / e.sum(axis=1, keepdims=True)).sum(axis=0)
+    return out
+
+
+def freekv_step(q_cur, q_prev, k, v, cu_seqlens, idx_prev, n_kv: int, w: int, pool_k: int, budget: int,
+                tau: float, dtype: str, scale: float | None = None, flags=None):
+    """One decode step.  Returns (flags, idx, k_c, v_c, out): the heads flagged
+    by freekv_flags (or the given flags) get a fresh index list from
+    decode_query_scores -> pool_prefix -> select_topk; the others keep
+    idx_prev; k_c / v_c are the rows idx names; out is gqa_decode of q_cur over
+    them."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lens = np.diff(cu)
+    if flags is None:
+        flags, _ = freekv_flags(q_cur, q_prev, n_kv, tau, dtype)
+    raw = decode_query_scores(q_cur, k, cu, n_kv, dtype, scale)
+    fresh = select_topk(pool_prefix(raw, cu, w, pool_k), cu, w, budget)
+    idx = np.array(idx_prev, dtype=np.int64, copy=True)
+    cb = budget_offsets(lens, budget)
+    for b in range(len(lens)):
+        for h in range(n_kv):
+            if flags[b, h]:
+                idx[h, cb[b]:cb[b + 1]] = fresh[h, cb[b]:cb[b + 1]]
+    k_c, v_c = gather_kv(k, v, idx, cu, budget)
+    out = gqa_decode(q_cur, k_c, v_c, cb[:-1], np.diff(cb), n_kv, dtype, scale)
+    return flags, idx, k_c, v_c, out

@@ -60,6 +60,14 @@ def test_budget_offsets(L):
         kvc.kvc_budget_offsets([5, -1], 3)
 
 
+def test_pyramid_budgets_host_helper(L):
+    for args in [(32, 3276, 1000), (32, 2048, 2048), (1, 500, 100), (7, 300, 32), (2, 64, 0)]:
+        np.testing.assert_array_equal(kvc.kvc_pyramid_budgets(*args), O.pyramid_budgets(*args))
+    for bad in [(0, 10, 5), (4, 10, 11), (4, 10, -1)]:
+        with pytest.raises(kvc.KvcError):
+            kvc.kvc_pyramid_budgets(*bad)
+
+
 def test_workspace_sizes(L):
     sl = np.array([32768], dtype=np.int32)
     n = kvc.kvc_score_window_workspace_size(kvc.KVC_BF16, sl, 32, 8, 128, 32)

@@ -88,6 +88,45 @@ def test_fastkv_tsp_layer_and_next_layer():
     run_and_check_compress("bf16", [k_tsp + W], N_H, N_KV, D, W, POOL, kv_budget, seed=1004 + 16, boost_frac=0.01)
 
 
+@pytest.mark.parametrize("schedule", ["uniform", "pyramid"])
+def test_fastkv_32_layer_chain(schedule):
+    """The whole FastKV workload: 32 layers of the Llama-3-8B shape, layers
+    0-15 at S = 32768, token-selective propagation at layer 15 (k_tsp =
+    floor(0.2 S) plus the window, hidden [S, 4096]), layers 16-31 at
+    S' = k_tsp + 32.  Per-layer KV budgets: 10% of S on every layer, or the
+    PyramidKV schedule around the same mean (first layer 2 * 3276 - 1024,
+    last layer 1024).  Every layer's one-call compression is checked against
+    the oracle."""
+    from kv_cache_compression_score_b200 import kvc
+    S, L = 32768, 32
+    k_tsp, b_avg = O.rate_count(0.2, S), O.rate_count(0.1, S)
+    budgets = (np.full(L, b_avg) if schedule == "uniform" else kvc.kvc_pyramid_budgets(L, b_avg, 1024))
+    if schedule == "pyramid":
+        np.testing.assert_array_equal(budgets, O.pyramid_budgets(L, b_avg, 1024))
+    S_next = k_tsp + W
+    n_diff = 0
+    for layer in range(L):
+        length = S if layer <= 15 else S_next
+        r = run_and_check_compress("bf16", [length], N_H, N_KV, D, W, POOL, int(budgets[layer]),
+                                   seed=4000 + layer, boost_frac=0.01, fused_call=True)
+        n_diff += r["n_diff"]
+        if layer == 15:
+            hidden = synth.hidden_states(4100, S, 4096, "bf16")
+            sel = TspSelector(S, W, POOL, k_tsp, 4096, "bf16")
+            idx, hout = sel.run(r["comp"].buf.scores_raw, to_device(hidden, "bf16"))
+            torch.cuda.synchronize()
+            g = idx.cpu().numpy()
+            idx_o = O.tsp_select(r["raw_o"], S, W, POOL, k_tsp)
+            pooled_o = O.tsp_pooled(r["raw_o"], S, W, POOL)
+            kth = np.sort(pooled_o)[::-1][k_tsp - 1]
+            diff = set(g[:k_tsp].tolist()) ^ set(idx_o[:k_tsp].tolist())
+            assert all(abs(pooled_o[j] - kth) <= 1e-5 * kth for j in diff)
+            assert np.array_equal(from_device(hout), O.tsp_gather(hidden, g))
+        del r
+    log_parity(dict(what="fastkv_chain", schedule=schedule, layers=L, budgets=[int(b) for b in budgets],
+                    tie_band_index_differences=n_diff))
+
+
 @pytest.mark.parametrize("fused", [False, True])
 def test_ragged_16_sequences(fused):
     lens = synth.ragged_lengths(1005, 16, 4096, 65536)

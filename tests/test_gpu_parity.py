@@ -208,7 +208,8 @@ def test_gather_isolated_bit_exact(dtype, d):
 
 # ------------------------------------------------------------------ decode
 @pytest.mark.parametrize("dtype,d,n_h,n_kv", [("f32", 64, 4, 2), ("bf16", 128, 32, 8), ("bf16", 64, 8, 8),
-                                              ("f32", 128, 16, 2)])
+                                              ("f32", 128, 16, 2), ("bf16", 128, 16, 8), ("bf16", 128, 64, 8),
+                                              ("bf16", 64, 16, 4)])
 def test_decode_isolated(dtype, d, n_h, n_kv):
     """Synthetic compact caches with ragged lengths, one empty cache, a
     length-1 cache and two queries aliasing the same cache."""

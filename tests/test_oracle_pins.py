@@ -488,3 +488,87 @@ def test_decode_q8_lossless_cache_equals_plain_decode():
     got = O.gqa_decode_q8(q, kq, vq, ks.T, vs.T, offs, lens, n_kv, "bf16")
     ref = O.gqa_decode(q, kf, vf, offs, lens, n_kv, "bf16", cache_dtype="f32")
     np.testing.assert_allclose(got, ref, rtol=1e-14, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# PyramidKV per-layer budgets
+# ---------------------------------------------------------------------------
+def test_pyramid_budgets_shape_and_mean():
+    b = O.pyramid_budgets(32, 3276, 1000)
+    assert b[0] == 2 * 3276 - 1000 and b[-1] == 1000          # the two ends
+    assert np.all(np.diff(b) <= 0)                            # never grows with depth
+    steps = -np.diff(b)
+    assert steps.max() - steps.min() <= 1                     # linear up to rounding
+    assert 32 * 3276 <= b.sum() < 32 * 3276 + 32              # mean B_avg, rounded up by < 1 per layer
+    np.testing.assert_array_equal(O.pyramid_budgets(8, 100, 100), np.full(8, 100))   # flat schedule
+    np.testing.assert_array_equal(O.pyramid_budgets(1, 77, 10), [77])
+    np.testing.assert_array_equal(O.pyramid_budgets(3, 10, 4), [16, 10, 4])           # by hand
+    np.testing.assert_array_equal(O.pyramid_budgets(4, 10, 5), [15, 12, 9, 5])        # 15 - floor(10 l / 3)
+    with pytest.raises(ValueError):
+        O.pyramid_budgets(4, 10, 11)
+
+
+# ---------------------------------------------------------------------------
+# FreeKV decode-time retrieval
+# ---------------------------------------------------------------------------
+def test_freekv_cosine_cases_by_hand():
+    """Hand-made query pairs: equal (cos 1), opposite (-1), orthogonal (0),
+    45 degrees (1/sqrt 2), a zero vector (0 by convention)."""
+    d = 4
+    cur = np.array([[[1, 0, 0, 0], [0, 2, 0, 0], [1, 0, 0, 0], [3, 0, 0, 0], [0, 0, 0, 0], [1, 1, 0, 0]]],
+                   dtype=np.float32)
+    prev = np.array([[[2, 0, 0, 0], [0, -1, 0, 0], [0, 0, 5, 0], [1, 1, 0, 0], [1, 0, 0, 0], [1, 1, 0, 0]]],
+                    dtype=np.float32)
+    flags, cos = O.freekv_flags(cur, prev, 3, 0.5, "f32")        # G = 2: heads (0,1), (2,3), (4,5)
+    np.testing.assert_allclose(cos[0], [1, -1, 0, 1 / math.sqrt(2), 0, 1], rtol=1e-15, atol=1e-15)
+    np.testing.assert_array_equal(flags[0], [True, True, True])     # group minima -1, 0, 0
+    flags, _ = O.freekv_flags(cur, prev, 6, 0.5, "f32")             # G = 1
+    np.testing.assert_array_equal(flags[0], [False, True, True, False, True, False])
+    assert d == cur.shape[-1]
+
+
+def test_decode_query_scores_is_a_one_row_window():
+    """A decode query after the cache scores keys exactly as an observation
+    window of one row placed on the last cached position (which sees every
+    key), and torch's fp64 softmax agrees."""
+    lengths, n_h, n_kv, d = [30, 9], 4, 2, 8
+    bt = _batch(lengths, n_h, n_kv, d, 1, seed=61, dtype="bf16")
+    q = bt["q_win"].reshape(len(lengths), n_h, d)                  # one window row per sequence
+    raw = O.decode_query_scores(q, bt["k"], bt["cu_seqlens"], n_kv, "bf16")
+    raw_w = O.raw_scores(bt["q_win"], bt["k"], bt["cu_seqlens"], n_h, n_kv, 1, "bf16")
+    np.testing.assert_allclose(raw, raw_w, rtol=1e-13, atol=1e-300)
+    G = n_h // n_kv
+    qt = torch.tensor(O.to_f64(q, "bf16"))
+    kt = torch.tensor(O.to_f64(bt["k"], "bf16"))
+    z = torch.einsum("gd,jd->gj", qt[0, 0:G], kt[0:30, 0]) / math.sqrt(d)
+    np.testing.assert_allclose(raw[0, 0:30], torch.softmax(z, dim=1).sum(0).numpy(), rtol=1e-13)
+    # K = 0: every key gets G / len
+    raw0 = O.decode_query_scores(q, np.zeros_like(bt["k"]), bt["cu_seqlens"], n_kv, "bf16")
+    np.testing.assert_allclose(raw0[:, :30], G / 30, rtol=1e-14)
+    np.testing.assert_allclose(raw0[:, 30:], G / 9, rtol=1e-14)
+
+
+def test_freekv_step_tau_extremes():
+    """tau = -2: no head is corrected, the step is decode over the previous
+    compact cache; tau = 2: every head is corrected, the step is a fresh
+    score / select / gather with the current query followed by decode."""
+    lengths, n_h, n_kv, d, w, B = [60, 45], 8, 2, 16, 4, 20
+    bt = _batch(lengths, n_h, n_kv, d, w, seed=71, dtype="bf16")
+    cu = bt["cu_seqlens"]
+    q_prev = synth.decode_queries(72, 2, n_h, d, "bf16")
+    q_cur = synth.decode_queries(73, 2, n_h, d, "bf16")
+    idx_prev = O.select_topk(O.pool_prefix(O.decode_query_scores(q_prev, bt["k"], cu, n_kv, "bf16"), cu, w, 5),
+                             cu, w, B)
+    f, idx, kc, vc, out = O.freekv_step(q_cur, q_prev, bt["k"], bt["v"], cu, idx_prev, n_kv, w, 5, B, -2.0, "bf16")
+    assert not f.any()
+    np.testing.assert_array_equal(idx, idx_prev)
+    kc_p, vc_p = O.gather_kv(bt["k"], bt["v"], idx_prev, cu, B)
+    cb = O.budget_offsets(lengths, B)
+    np.testing.assert_array_equal(out, O.gqa_decode(q_cur, kc_p, vc_p, cb[:-1], np.diff(cb), n_kv, "bf16"))
+    f, idx, kc, vc, out = O.freekv_step(q_cur, q_prev, bt["k"], bt["v"], cu, idx_prev, n_kv, w, 5, B, 2.0, "bf16")
+    assert f.all()
+    fresh = O.select_topk(O.pool_prefix(O.decode_query_scores(q_cur, bt["k"], cu, n_kv, "bf16"), cu, w, 5), cu, w, B)
+    np.testing.assert_array_equal(idx, fresh)
+    # the same query twice: cos = 1, nothing below tau = 0.999
+    f, idx, _, _, _ = O.freekv_step(q_cur, q_cur, bt["k"], bt["v"], cu, idx_prev, n_kv, w, 5, B, 0.999, "bf16")
+    assert not f.any() and np.array_equal(idx, idx_prev)
