@@ -316,6 +316,46 @@ kvc_status kvc_gqa_decode_attn_q8(int batch, int n_h, int n_kv, int d_h, float s
                                   const int64_t *kv_row_offset, const int32_t *kv_len, int max_kv_len,
                                   float *out, void *ws, size_t ws_bytes, kvc_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * FreeKV decode step with fine-grained correction.  Source: "FreeKV: Boosting
+ * KV Cache Retrieval for Efficient LLM Inference", technical summary section
+ * 2.A ("Recuperation Speculative": a step reuses the tokens retrieved for the
+ * previous step; "Correction Fine": the heads whose query similarity to the
+ * previous step falls below tau are selected and retrieved again before
+ * attention).  All caches stay in device memory (the page's CPU offload is
+ * not part of this library).
+ *
+ * For sequence b and KV head h (query heads h*G .. h*G+G-1):
+ *   reselected[b][h] = 1 if min_g cos(q_cur[b][hG+g], q_prev[b][hG+g]) < tau
+ *                      (cos = 0 when a vector is zero), else 0;
+ *   if reselected: its index list is replaced by the budgeted selection (the
+ *     rule of kvc_select_topk: w most recent tokens kept, max-pooled prefix
+ *     scores, lowest position first on ties) over the scores
+ *     raw[j] = sum_g softmax_j(scale * q_cur[b][hG+g] . k_j), j < len_b (the
+ *     decode query sees every cached key), max-pooled over [0, len_b - w);
+ *     its rows of k_c / v_c are gathered again;
+ *   otherwise idx, k_c and v_c keep their contents for that head;
+ *   out[b] = kvc_gqa_decode_attn of q_cur[b] over the compact cache rows
+ *     [cu_budget[b], cu_budget[b+1]) of every head.
+ * Heads whose flag is 0 read no full-cache key.
+ *
+ * bf16 only; d_h in {64, 128}; G in {1, 2, 4, 8}.  q_cur, q_prev: [batch,
+ * n_h, d_h]; k, v: full caches [T, n_kv, d_h] (cu_seqlens, len_b >= w);
+ * cu_budget from kvc_budget_offsets(budget); idx: int32 [n_kv,
+ * cu_budget[batch]] and k_c, v_c: [cu_budget[batch], n_kv, d_h], in/out
+ * (hold the previous step's selection; on the first step pass tau > 1 so
+ * that every head is selected); reselected: int32 [batch, n_kv], out;
+ * out: float32 [batch, n_h, d_h].  ws: kvc_freekv_workspace_size() bytes,
+ * zeroed before its first use (decode counters, left zero by every call).
+ * ------------------------------------------------------------------------ */
+size_t kvc_freekv_workspace_size(int batch, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w,
+                                 int budget);
+kvc_status kvc_freekv_step(int batch, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                           const int32_t *cu_budget, int n_h, int n_kv, int d_h, int w, int pool_k, int budget,
+                           float tau, float scale, const void *q_cur, const void *q_prev, const void *k,
+                           const void *v, int32_t *idx, void *k_c, void *v_c, int32_t *reselected, float *out,
+                           void *ws, size_t ws_bytes, kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -530,6 +530,114 @@ kvc_status kvc_gqa_decode_attn_q8(int batch, int n_h, int n_kv, int d_h, float s
   return KVC_OK;
 }
 
+// ------------------------------------------------------------------ FreeKV
+namespace {
+struct FreeKvPlan {
+  DecodePlan dec;
+  int n_chunks = 0, G = 0, max_kept = 0;
+  int64_t zpitch = 0, total_kept = 0;
+  Batch bt;
+  size_t off_dec = 0, off_flags = 0, off_doff = 0, off_dlen = 0, off_part = 0, off_scores = 0, off_z = 0, bytes = 0;
+};
+
+kvc_status plan_freekv(int batch, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w, int budget,
+                       FreeKvPlan *pl) {
+  kvc_status s = check_batch(batch, seqlens_host, w, &pl->bt);
+  if (s != KVC_OK) return s;
+  if (w < 1) return fail(KVC_ERR_INVALID_ARG, "w must be >= 1 (got %d)", w);
+  if (budget < w) return fail(KVC_ERR_INVALID_ARG, "budget (%d) must be >= w (%d): the window is always kept", budget, w);
+  int64_t total = 0;
+  int max_kept = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int kept = std::min(budget, seqlens_host[b]);
+    total += kept;
+    max_kept = std::max(max_kept, kept);
+  }
+  s = plan_decode(KVC_BF16, batch, n_h, n_kv, d_h, max_kept, &pl->dec);
+  if (s != KVC_OK) return s;
+  pl->G = n_h / n_kv;
+  pl->max_kept = max_kept;
+  pl->total_kept = total;
+  pl->n_chunks = (pl->bt.max_len + kvc::freekv_chunk_keys() - 1) / kvc::freekv_chunk_keys();
+  pl->zpitch = (int64_t)round_up((size_t)pl->bt.max_len, 4);
+  const size_t units = (size_t)batch * n_kv;
+  pl->off_dec = 0;                                             // the decode workspace (error word first)
+  pl->off_flags = round_up(pl->dec.bytes, 256);
+  pl->off_doff = round_up(pl->off_flags + units * sizeof(int), 256);
+  pl->off_dlen = round_up(pl->off_doff + (size_t)batch * sizeof(int64_t), 256);
+  pl->off_part = round_up(pl->off_dlen + (size_t)batch * sizeof(int), 256);
+  pl->off_scores = round_up(pl->off_part + units * pl->n_chunks * pl->G * sizeof(float2), 256);
+  pl->off_z = round_up(pl->off_scores + (size_t)n_kv * pl->bt.T * sizeof(float), 256);
+  pl->bytes = pl->off_z + units * pl->G * (size_t)pl->zpitch * sizeof(float);
+  return KVC_OK;
+}
+}  // namespace
+
+size_t kvc_freekv_workspace_size(int batch, const int32_t *seqlens_host, int n_h, int n_kv, int d_h, int w,
+                                 int budget) {
+  FreeKvPlan pl;
+  if (plan_freekv(batch, seqlens_host, n_h, n_kv, d_h, w, budget, &pl) != KVC_OK) return 0;
+  return pl.bytes;
+}
+
+kvc_status kvc_freekv_step(int batch, const int32_t *seqlens_host, const int32_t *cu_seqlens,
+                           const int32_t *cu_budget, int n_h, int n_kv, int d_h, int w, int pool_k, int budget,
+                           float tau, float scale, const void *q_cur, const void *q_prev, const void *k,
+                           const void *v, int32_t *idx, void *k_c, void *v_c, int32_t *reselected, float *out,
+                           void *ws, size_t ws_bytes, kvc_stream_t stream) {
+  FreeKvPlan pl;
+  kvc_status s = plan_freekv(batch, seqlens_host, n_h, n_kv, d_h, w, budget, &pl);
+  if (s != KVC_OK) return s;
+  if (pool_k < 1 || pool_k > 31 || pool_k % 2 == 0)
+    return fail(KVC_ERR_INVALID_ARG, "pool_k must be odd and in [1, 31] (got %d)", pool_k);
+  if (!cu_seqlens || !cu_budget) return fail(KVC_ERR_INVALID_ARG, "cu_seqlens / cu_budget is NULL");
+  if (!aligned16(q_cur) || !aligned16(q_prev) || !aligned16(k) || !aligned16(v) || !aligned16(idx) ||
+      !aligned16(k_c) || !aligned16(v_c) || !aligned16(reselected) || !aligned16(out))
+    return fail(KVC_ERR_INVALID_ARG, "q_cur, q_prev, k, v, idx, k_c, v_c, reselected and out must be non-NULL "
+                "and 16-byte aligned");
+  if (!aligned16(ws) || ws_bytes < pl.bytes)
+    return fail(KVC_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", pl.bytes, ws_bytes);
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_h);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  kvc::FreeKvArgs f;
+  f.q_cur = static_cast<const __nv_bfloat16 *>(q_cur);
+  f.q_prev = static_cast<const __nv_bfloat16 *>(q_prev);
+  f.k = static_cast<const __nv_bfloat16 *>(k);
+  f.cu_seqlens = cu_seqlens;
+  f.cu_budget = cu_budget;
+  f.flags = reselected;
+  f.dec_off = reinterpret_cast<int64_t *>(wsb + pl.off_doff);
+  f.dec_len = reinterpret_cast<int *>(wsb + pl.off_dlen);
+  f.z = reinterpret_cast<float *>(wsb + pl.off_z);
+  f.part = reinterpret_cast<float2 *>(wsb + pl.off_part);
+  f.scores = reinterpret_cast<float *>(wsb + pl.off_scores);
+  f.batch = batch; f.n_h = n_h; f.n_kv = n_kv; f.d_h = d_h; f.w = w; f.pool_r = pool_k / 2;
+  f.n_chunks = pl.n_chunks; f.T_total = (int)pl.bt.T; f.zpitch = pl.zpitch;
+  f.c = scale * 1.4426950408889634f;
+  f.tau = tau;
+  cudaError_t e = kvc::freekv_rescore(f, st);
+  if (e != cudaSuccess) return cuda_fail(e, "FreeKV re-scoring kernels");
+  e = kvc::select_topk(f.scores, idx, cu_seqlens, cu_budget, batch, n_kv, (int)pl.bt.T, (int)pl.total_kept, w, budget,
+                       std::max(pl.bt.max_len, w), st, reselected);
+  if (e != cudaSuccess) return cuda_fail(e, "FreeKV select kernel");
+  e = kvc::gather_rows_kv(k, v, k_c, v_c, idx, cu_seqlens, cu_budget, batch, n_kv, d_h * 2, (int)pl.total_kept,
+                          pl.max_kept, st, reselected);
+  if (e != cudaSuccess) return cuda_fail(e, "FreeKV gather kernel");
+  kvc::DecodeArgs a;
+  a.dt = KVC_BF16; a.batch = batch; a.n_h = n_h; a.n_kv = n_kv; a.d_h = d_h; a.scale = scale;
+  a.q = q_cur; a.k_c = k_c; a.v_c = v_c; a.row_off = f.dec_off; a.kv_len = f.dec_len; a.out = out;
+  a.tickets = reinterpret_cast<int *>(wsb + pl.off_dec + pl.dec.off_tickets);
+  a.err = reinterpret_cast<int *>(wsb);
+  a.cache_rows = std::max<int64_t>(1, pl.total_kept);
+  a.part = reinterpret_cast<float *>(wsb + pl.off_dec + pl.dec.off_part);
+  a.n_chunks = pl.dec.n_chunks;
+  a.chunk_rows = pl.dec.chunk_rows;
+  e = kvc::gqa_decode(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "FreeKV decode kernel");
+  return KVC_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

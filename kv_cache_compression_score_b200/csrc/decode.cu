@@ -66,11 +66,6 @@ template <typename T> KVC_DEVINL void unpack16(const uint4 &v, float *o);
 template <> KVC_DEVINL void unpack16<__nv_bfloat16>(const uint4 &v, float *o) { Elem<__nv_bfloat16>::unpack(v, o); }
 template <> KVC_DEVINL void unpack16<float>(const uint4 &v, float *o) { Elem<float>::unpack(v, o); }
 
-KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-
 // warp w's slice of the flattened row space is [start(w), start(w + 1))
 KVC_DEVINL int64_t slice_start(int64_t w, int64_t R, int64_t NW) { return w * R / NW; }
 // the warp whose slice contains global row x (0 <= x < R)

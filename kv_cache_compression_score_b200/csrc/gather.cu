@@ -18,7 +18,8 @@ constexpr int kGatherUnroll = 4;
 __global__ void __launch_bounds__(kGatherThreads)
 gather_kv_kernel(const uint8_t *__restrict__ k, const uint8_t *__restrict__ v, uint8_t *__restrict__ k_out,
                  uint8_t *__restrict__ v_out, const int32_t *__restrict__ idx, const int *__restrict__ cu_seqlens,
-                 const int *__restrict__ cu_budget, int n_kv, int vec_per_head, int total_budget) {
+                 const int *__restrict__ cu_budget, int n_kv, int vec_per_head, int total_budget,
+                 const int *__restrict__ mask) {
   grid_dependency_wait();
   allow_dependents();
   const int b = blockIdx.y;
@@ -40,6 +41,7 @@ gather_kv_kernel(const uint8_t *__restrict__ k, const uint8_t *__restrict__ v, u
         const int t = (int)(e / row_vecs);
         const int rem = (int)(e - (long long)t * row_vecs);
         const int h = rem / vec_per_head, c = rem - h * vec_per_head;
+        if (mask && !mask[b * n_kv + h]) { ok[u] = false; continue; }   // this head keeps its rows
         const int src_t = idx[(size_t)h * total_budget + cb + t];
         dst_off[u] = ((size_t)(cb + t) * n_kv + h) * head_bytes + (size_t)c * 16;
         if (src_t >= 0 && src_t < len) {
@@ -182,7 +184,8 @@ cudaError_t gather_rows_kv_q8(const void *k, const void *v, int8_t *kq, int8_t *
 
 cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_out, const int32_t *idx,
                            const int32_t *cu_seqlens, const int32_t *cu_budget, int n_seqs, int n_kv,
-                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st) {
+                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st,
+                           const int32_t *mask) {
   const int vph = row_bytes_per_head / 16;
   const long long items = (long long)max_kept * n_kv * vph;
   long long blocks = (items + kGatherThreads * kGatherUnroll - 1) / (kGatherThreads * kGatherUnroll);
@@ -192,7 +195,7 @@ cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_ou
   count_launch();
   return launch_pdl(gather_kv_kernel, grid, dim3(kGatherThreads), 0, st, static_cast<const uint8_t *>(k),
                     static_cast<const uint8_t *>(v), static_cast<uint8_t *>(k_out), static_cast<uint8_t *>(v_out), idx,
-                    cu_seqlens, cu_budget, n_kv, vph, total_budget);
+                    cu_seqlens, cu_budget, n_kv, vph, total_budget, mask);
 }
 
 cudaError_t gather_hidden(const void *hidden, void *out, const int32_t *idx, int n_rows, int row_bytes, int n_src,

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <cuda.h>
 
 #define KVC_DEVINL __device__ __forceinline__
 
@@ -185,6 +186,74 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
        | (1u << 10)                      // B format: bf16
        | ((uint32_t)(N >> 3) << 17)      // N / 8
        | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor copies (no multicast), cp.async, ldmatrix / mma.sync / movmatrix
+// for the small-N products of the decode-shaped kernels
+// ---------------------------------------------------------------------------
+KVC_DEVINL void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+               :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+KVC_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y) : "memory");
+}
+KVC_DEVINL void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" :: "l"(map) : "memory");
+}
+// 16-byte cp.async, zero-filled (no global read) when !valid
+KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+KVC_DEVINL void cp_async4(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+// arrive on *bar once every cp.async this thread issued so far has landed
+// (the arrival counts against the barrier's expected count)
+KVC_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+KVC_DEVINL void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+KVC_DEVINL void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+KVC_DEVINL void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+               "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+KVC_DEVINL uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// (lo, hi) -> bf16x2 with lo in the low half, round to nearest even
+KVC_DEVINL uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// byte offset of 16-byte chunk `ch` of row `r` inside a tile whose rows are
+// cut into boxes of BoxB bytes (BoxB-byte swizzle: the chunk index is XORed
+// with address bits 7.. of the row start)
+template <int BoxB, int Rows>
+KVC_DEVINL uint32_t swz(int r, int ch) {
+  constexpr int kCh = BoxB / 16;                    // chunks per box row
+  const int box = ch / kCh, c = ch % kCh;
+  const int x = BoxB == 128 ? (r & 7) : ((r >> 1) & 3);
+  return (uint32_t)(box * Rows * BoxB + r * BoxB + ((c ^ x) << 4));
 }
 
 // ---------------------------------------------------------------------------

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "kvc.h"
@@ -50,13 +51,34 @@ int tc_select_max_keys(int d_h);  // fused selection: largest key chunk it keeps
 cudaError_t pool_prefix(const float *raw, float *scores, const int32_t *cu_seqlens, int n_seqs, int n_kv,
                         int T_total, int max_len, int w, int pool_k, cudaStream_t st);
 
+// mask (nullable): int32 [n_seqs * n_kv]; (sequence, head) pairs whose entry
+// is 0 are left untouched
 cudaError_t select_topk(const float *scores, int32_t *idx, const int32_t *cu_seqlens, const int32_t *cu_budget,
                         int n_seqs, int n_kv, int T_total, int total_budget, int w, int budget, int max_len,
-                        cudaStream_t st);
+                        cudaStream_t st, const int32_t *mask = nullptr);
 
 cudaError_t gather_rows_kv(const void *k, const void *v, void *k_out, void *v_out, const int32_t *idx,
                            const int32_t *cu_seqlens, const int32_t *cu_budget, int n_seqs, int n_kv,
-                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st);
+                           int row_bytes_per_head, int total_budget, int max_kept, cudaStream_t st,
+                           const int32_t *mask = nullptr);
+
+// FreeKV re-scoring of the drifted heads (freekv.cu)
+struct FreeKvArgs {
+  const __nv_bfloat16 *q_cur, *q_prev, *k;
+  const int *cu_seqlens, *cu_budget;
+  int *flags;            // [batch * n_kv] 1: scored and selected again this step
+  int64_t *dec_off;      // [batch] decode row offsets of the compact caches
+  int *dec_len;          // [batch] decode lengths
+  float *z;              // [batch, n_kv, G, zpitch] logits (log2 units)
+  float2 *part;          // [batch, n_kv, n_chunks, G] (max, sum of 2^(z - max)) per key chunk
+  float *scores;         // [n_kv, T_total] pooled scores of the flagged heads
+  int batch, n_h, n_kv, d_h, w, pool_r, n_chunks, T_total;
+  int64_t zpitch;
+  float c;               // scale * log2(e)
+  float tau;
+};
+cudaError_t freekv_rescore(const FreeKvArgs &a, cudaStream_t st);
+int freekv_chunk_keys();
 
 cudaError_t gather_rows_kv_q8(const void *k, const void *v, int8_t *kq, int8_t *vq, float *ks, float *vs,
                               int64_t scale_pitch, const int32_t *idx, const int32_t *cu_seqlens,

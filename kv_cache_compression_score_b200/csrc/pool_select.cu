@@ -529,10 +529,12 @@ KVC_DEVINL void cluster_topk_ascending(const float *__restrict__ src, int n, int
 
 __global__ void __launch_bounds__(kCThreads)
 select_topk_cluster(const float *__restrict__ scores, int32_t *__restrict__ idx, const int *__restrict__ cu_seqlens,
-                    const int *__restrict__ cu_budget, int T_total, int total_budget, int w, int budget) {
+                    const int *__restrict__ cu_budget, int T_total, int total_budget, int w, int budget,
+                    const int *__restrict__ mask) {
   grid_dependency_wait();
   allow_dependents();
   const int h = blockIdx.x / kClu, b = blockIdx.y;
+  if (mask && !mask[b * (gridDim.x / kClu) + h]) return;   // the same decision in every CTA of the cluster
   const uint32_t rank = cluster_rank();
   const int t0 = cu_seqlens[b], len = cu_seqlens[b + 1] - t0;
   int32_t *dst = idx + (size_t)h * total_budget + cu_budget[b];
@@ -613,9 +615,9 @@ static size_t cluster_cache_bytes(int n) {
 
 cudaError_t select_topk(const float *scores, int32_t *idx, const int32_t *cu_seqlens, const int32_t *cu_budget,
                         int n_seqs, int n_kv, int T_total, int total_budget, int w, int budget, int max_len,
-                        cudaStream_t st) {
+                        cudaStream_t st, const int32_t *mask) {
   void *args[] = {(void *)&scores, (void *)&idx, (void *)&cu_seqlens, (void *)&cu_budget, (void *)&T_total,
-                  (void *)&total_budget, (void *)&w, (void *)&budget};
+                  (void *)&total_budget, (void *)&w, (void *)&budget, (void *)&mask};
   return launch_cluster((const void *)select_topk_cluster, dim3(kClu * n_kv, n_seqs), cluster_cache_bytes(max_len - w),
                         st, args);
 }

@@ -126,18 +126,6 @@ struct TcWork {
   int b, h, c, t0, len, P, key_begin, key_end, n_tiles;
 };
 
-// 16-byte cp.async, zero-filled (no global read) when !valid
-KVC_DEVINL void cp_async16(void *dst, const void *src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-               :: "r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-
-// arrive on *bar once every cp.async this thread issued so far has landed
-// (the arrival counts against the barrier's expected count)
-KVC_DEVINL void cp_async_arrive_noinc(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-
 // Q_win rows r = g * w + i of (b, h) into the 128-byte-swizzled K-major tile
 // with cp.async (all chunks in flight at once); rows >= R are zero-filled.
 // The caller makes their completion arrive on q_full.

@@ -50,6 +50,9 @@ SIGNATURES = {
                                   _c_p, _c_p, _c_i64, _c_p]),
     "kvc_gqa_decode_attn_q8": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i64,
                                         _c_i64, _c_p, _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
+    "kvc_freekv_workspace_size": (_c_sz, [_c_int, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "kvc_freekv_step": (_c_int, [_c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_f,
+                                 _c_f, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "kvc_gqa_decode_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_i64, _c_p,
                                      _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
@@ -242,3 +245,18 @@ def kvc_gqa_decode_attn_q8(q, k_q, v_q, k_scale, v_scale, kv_row_offset, kv_len,
                                         _dptr(k_scale), _dptr(v_scale), k_scale.shape[1], k_q.shape[0],
                                         _dptr(kv_row_offset), _dptr(kv_len), max_kv_len, _dptr(out), _dptr(ws),
                                         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_freekv_workspace_size(seqlens, n_h: int, n_kv: int, d_h: int, w: int, budget: int) -> int:
+    sl, p = _host_i32(seqlens)
+    return int(lib().kvc_freekv_workspace_size(len(sl), p, n_h, n_kv, d_h, w, budget))
+
+
+def kvc_freekv_step(seqlens, cu_seqlens, cu_budget, n_h: int, w: int, pool_k: int, budget: int, tau: float,
+                    scale: float, q_cur, q_prev, k, v, idx, k_c, v_c, reselected, out, ws, stream=None) -> None:
+    """One FreeKV decode step: re-select the heads whose query drifted, then decode."""
+    sl, p = _host_i32(seqlens)
+    _check(lib().kvc_freekv_step(len(sl), p, _dptr(cu_seqlens), _dptr(cu_budget), n_h, k.shape[1], k.shape[2], w,
+                                 pool_k, budget, tau, scale, _dptr(q_cur), _dptr(q_prev), _dptr(k), _dptr(v),
+                                 _dptr(idx), _dptr(k_c), _dptr(v_c), _dptr(reselected), _dptr(out), _dptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))

@@ -144,3 +144,33 @@ class TspSelector:
         kvc.kvc_tsp_select_gather(scores_raw, self.w, self.pool_k, self.k_tsp, hidden, self.idx, self.hidden_out,
                                   self.ws, stream)
         return self.idx, self.hidden_out
+
+
+class FreeKvStep:
+    """FreeKV decode steps over full caches of one packed batch (kvc_freekv_step):
+    holds the index lists, compact caches, flags and output between steps."""
+
+    def __init__(self, seqlens, n_h: int, n_kv: int, d_h: int, w: int, pool_k: int, budget: int, tau: float,
+                 scale: float = 0.0, device="cuda"):
+        self.n_h, self.w, self.pool_k, self.budget, self.tau, self.scale = n_h, w, pool_k, budget, tau, scale
+        sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+        cu = np.zeros(len(sl) + 1, dtype=np.int32)
+        cu[1:] = np.cumsum(sl)
+        cb = kvc.kvc_budget_offsets(sl, budget)
+        Tb = int(cb[-1])
+        self.seqlens = sl
+        self.cu_seqlens = torch.from_numpy(cu).to(device)
+        self.cu_budget_host = cb
+        self.cu_budget = torch.from_numpy(cb).to(device)
+        self.idx = torch.zeros((n_kv, Tb), dtype=torch.int32, device=device)
+        self.k_c = torch.zeros((Tb, n_kv, d_h), dtype=torch.bfloat16, device=device)
+        self.v_c = torch.zeros_like(self.k_c)
+        self.reselected = torch.zeros((len(sl), n_kv), dtype=torch.int32, device=device)
+        self.out = torch.empty((len(sl), n_h, d_h), dtype=torch.float32, device=device)
+        self.ws = zeroed_workspace(kvc.kvc_freekv_workspace_size(sl, n_h, n_kv, d_h, w, budget), device)
+
+    def step(self, q_cur, q_prev, k, v, tau=None, stream=None):
+        kvc.kvc_freekv_step(self.seqlens, self.cu_seqlens, self.cu_budget, self.n_h, self.w, self.pool_k, self.budget,
+                            self.tau if tau is None else tau, self.scale, q_cur, q_prev, k, v, self.idx, self.k_c,
+                            self.v_c, self.reselected, self.out, self.ws, stream)
+        return self.out

@@ -27,7 +27,7 @@ MASK64 = np.uint64(0xFFFFFFFFFFFFFFFF)
 GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
 
 # Tensor ids: one independent stream per (seed, id, sequence).
-T_QWIN, T_K, T_V, T_QDEC, T_HIDDEN, T_BOOST_DIR, T_BOOST_POS, T_LENGTHS, T_SCORES = range(1, 10)
+T_QWIN, T_K, T_V, T_QDEC, T_HIDDEN, T_BOOST_DIR, T_BOOST_POS, T_LENGTHS, T_SCORES, T_DRIFT = range(1, 11)
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -187,3 +187,18 @@ def index_lists(seed: int, lengths, n_kv: int, budget: int) -> np.ndarray:
             keys = uniform_u64(stream_key(seed, T_SCORES, b * 256 + h + 1), int(L))
             rows[h].append(np.sort(np.argsort(keys, kind="stable")[:kept]))
     return np.stack([np.concatenate(r) if r else np.zeros(0, np.int64) for r in rows]).astype(np.int32)
+
+
+def drifted_queries(seed: int, q_prev_bits: np.ndarray, dtype: str, lo: float = 0.0, hi: float = 0.9,
+                    group: int = 1) -> np.ndarray:
+    """Next-step decode queries: q_prev + sigma * noise with one sigma per
+    (batch entry, group of `group` consecutive query heads) drawn uniformly
+    from [lo, hi] -- from nearly equal queries to strongly drifted ones, so
+    that some groups fall below a similarity threshold and others do not."""
+    prev = bf16_bits_to_f32(q_prev_bits).astype(np.float64) if dtype == "bf16" else \
+        np.asarray(q_prev_bits, dtype=np.float64)
+    batch, n_h, d = prev.shape
+    sig = lo + (hi - lo) * uniform01(stream_key(seed, T_DRIFT, 0), batch * (n_h // group))
+    sig = np.repeat(sig.reshape(batch, n_h // group), group, axis=1).reshape(batch, n_h, 1)
+    noise = normal_f64(stream_key(seed, T_DRIFT, 1), batch * n_h * d).reshape(batch, n_h, d)
+    return round_to(prev + sig * noise, dtype)
