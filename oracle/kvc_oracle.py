@@ -43,6 +43,13 @@ or bf16 bit patterns, both widened exactly):
    a KV head whose query has drifted -- cosine similarity between the current
    and the previous query below tau -- is scored again with the current
    query, its tokens are selected again and retrieved before attention.
+12. ``xkv_factorize`` / ``xkv_reconstruct`` -- xKV cross-layer factorisation
+   and selective reconstruction (xKV, sections 2.2 and 2.3): the keys of a
+   window of W consecutive layers, concatenated along the feature axis, get a
+   rank-r truncated SVD X ~ U_r S_r V_r^T; the window keeps the shared token
+   basis A = U_r S_r = X V_r and one reconstruction block B_l (rows l*d ..
+   (l+1)*d of V_r, transposed) per layer; selective reconstruction rebuilds
+   only the chosen rows, K_l[idx] ~ A[idx] B_l.
 10. ``pyramid_budgets`` -- PyramidKV's per-layer cache budgets (attention-variants
    page, section "Compresser un cache existant": different layers get different
    budgets): a budget that falls linearly from the first layer to the last
@@ -78,6 +85,11 @@ Readings of points the pages leave open:
   w most recent tokens always kept) then pick its tokens.  Heads above tau
   keep their index list (and compact rows); decode attention then runs over
   every head's compact cache;
+* xKV: the factorisation is per (sequence, KV head) -- X_h = [K_1[:, h] | ...
+  | K_W[:, h]] of shape [S, W * d_h] -- and applies to the keys (values
+  alike); the chosen rows are an input (an index list per KV head, e.g. the
+  library's budgeted selection); reconstructed rows are stored as bf16
+  (round to nearest even) for decode;
 * quantised cache: symmetric int8 per (row, head) vector, scale = max|x| / 127
   and code = round-half-even(x / scale), both quotients in float32 (the
   precision the stored values have), codes clipped to [-127, 127]; an all-zero
@@ -470,3 +482,40 @@ def freekv_step(q_cur, q_prev, k, v, cu_seqlens, idx_prev, n_kv: int, w: int, po
     k_c, v_c = gather_kv(k, v, idx, cu, budget)
     out = gqa_decode(q_cur, k_c, v_c, cb[:-1], np.diff(cb), n_kv, dtype, scale)
     return flags, idx, k_c, v_c, out
+
+
+# ----------------------------------------------------------------------------
+# 12. xKV cross-layer factorisation and selective reconstruction
+# ----------------------------------------------------------------------------
+def xkv_factorize(k_layers, r: int, dtype: str):
+    """k_layers: W caches [S, n_kv, d] (stored).  Returns (A [n_kv, S, r],
+    Vt [n_kv, r, W * d]) in float64 with A = X_h V_r and Vt = V_r^T from the
+    truncated SVD of X_h = [K_1[:, h] | ... | K_W[:, h]]."""
+    X = np.concatenate([to_f64(k, dtype) for k in k_layers], axis=2)     # [S, n_kv, W d]
+    S, n_kv, Wd = X.shape
+    if not 1 <= r <= min(S, Wd):
+        raise ValueError("need 1 <= r <= min(S, W * d)")
+    A = np.zeros((n_kv, S, r))
+    Vt = np.zeros((n_kv, r, Wd))
+    for h in range(n_kv):
+        _, _, vt = np.linalg.svd(X[:, h, :], full_matrices=False)
+        Vt[h] = vt[:r]
+        A[h] = X[:, h, :] @ vt[:r].T
+    return A, Vt
+
+
+def xkv_reconstruct(A: np.ndarray, Vt: np.ndarray, layer: int, d: int, idx: np.ndarray) -> np.ndarray:
+    """Rows idx[h] of layer `layer` for every KV head: [n_sel, n_kv, d] float64,
+    row t of head h = A[h, idx[h, t]] @ Vt[h][:, layer*d:(layer+1)*d]."""
+    n_kv, n_sel = idx.shape
+    out = np.zeros((n_sel, n_kv, d))
+    for h in range(n_kv):
+        out[:, h, :] = A[h][np.asarray(idx[h], dtype=np.int64)] @ Vt[h][:, layer * d:(layer + 1) * d]
+    return out
+
+
+def xkv_window_bytes(S: int, n_kv: int, d: int, W: int, r: int, b_basis: int, b_blocks: int) -> int:
+    """Bytes one factorised window stores (per KV head: the S x r basis and the
+    r x (W d) reconstruction blocks), against W * S * n_kv * d * b for the
+    plain keys of the window."""
+    return n_kv * (S * r * b_basis + r * W * d * b_blocks)

@@ -572,3 +572,60 @@ def test_freekv_step_tau_extremes():
     # the same query twice: cos = 1, nothing below tau = 0.999
     f, idx, _, _, _ = O.freekv_step(q_cur, q_cur, bt["k"], bt["v"], cu, idx_prev, n_kv, w, 5, B, 0.999, "bf16")
     assert not f.any() and np.array_equal(idx, idx_prev)
+
+
+# ---------------------------------------------------------------------------
+# xKV cross-layer factorisation and selective reconstruction
+# ---------------------------------------------------------------------------
+def _low_rank_layers(seed, S, n_kv, d, W, rank, noise=0.0):
+    """W layers whose keys share a rank-`rank` token basis (plus noise).  The
+    factors are small integers, so without noise the stored float32 keys have
+    exactly that rank."""
+    U = np.round(2 * synth.normal_tensor(seed, synth.T_K, 0, (n_kv, S, rank), "f32").astype(np.float64))
+    layers = []
+    for l in range(W):
+        M = np.round(2 * synth.normal_tensor(seed, synth.T_V, l + 1, (n_kv, rank, d), "f32").astype(np.float64))
+        E = synth.normal_tensor(seed, synth.T_QDEC, l + 1, (n_kv, S, d), "f32").astype(np.float64)
+        layers.append(np.transpose(U @ M + noise * E, (1, 0, 2)).astype(np.float32))   # [S, n_kv, d]
+    return layers
+
+
+def test_xkv_exact_for_low_rank_windows():
+    """Keys of exact rank <= r are rebuilt exactly (Eckart-Young with no tail)."""
+    S, n_kv, d, W, r = 60, 2, 8, 3, 5
+    layers = _low_rank_layers(3, S, n_kv, d, W, 4)
+    A, Vt = O.xkv_factorize(layers, r, "f32")
+    idx = np.stack([np.arange(S)[::-1], np.arange(S)])
+    for l in range(W):
+        rec = O.xkv_reconstruct(A, Vt, l, d, idx)
+        for h in range(n_kv):
+            np.testing.assert_allclose(rec[:, h], layers[l][idx[h], h].astype(np.float64), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(np.einsum("hrk,hsk->hrs", Vt, Vt), np.broadcast_to(np.eye(r), (n_kv, r, r)),
+                               atol=1e-12)
+
+
+def test_xkv_error_is_the_singular_tail():
+    """Noisy window: the reconstruction error of all rows equals the norm of
+    the discarded singular values, and a single layer (W = 1) is the plain
+    truncated SVD of that layer."""
+    S, n_kv, d, W, r = 80, 2, 6, 4, 7
+    layers = _low_rank_layers(5, S, n_kv, d, W, 5, noise=0.3)
+    A, Vt = O.xkv_factorize(layers, r, "f32")
+    idx = np.broadcast_to(np.arange(S), (n_kv, S))
+    X = np.concatenate([l.astype(np.float64) for l in layers], axis=2)
+    rec = np.concatenate([O.xkv_reconstruct(A, Vt, l, d, idx) for l in range(W)], axis=2)
+    for h in range(n_kv):
+        sv = np.linalg.svd(X[:, h], compute_uv=False)
+        np.testing.assert_allclose(np.linalg.norm(X[:, h] - rec[:, h]), np.sqrt(np.sum(sv[r:] ** 2)), rtol=1e-9)
+    r1 = 4
+    A1, Vt1 = O.xkv_factorize(layers[:1], r1, "f32")
+    for h in range(n_kv):
+        u, sv, vt = np.linalg.svd(layers[0][:, h].astype(np.float64), full_matrices=False)
+        np.testing.assert_allclose(A1[h] @ Vt1[h], (u[:, :r1] * sv[:r1]) @ vt[:r1], atol=1e-9)
+
+
+def test_xkv_window_bytes():
+    # per head S*r basis + r*W*d blocks; 8x smaller than the window's keys for S=32768, d=128, W=4, r=64 (fp32 basis
+    # against bf16 keys: 4x)
+    assert O.xkv_window_bytes(32768, 8, 128, 4, 64, 4, 4) == 8 * (32768 * 64 * 4 + 64 * 512 * 4)
+    assert 4 * 32768 * 8 * 128 * 2 / O.xkv_window_bytes(32768, 8, 128, 4, 64, 2, 4) > 7.5
