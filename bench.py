@@ -578,6 +578,38 @@ def run_workloads(args, dev, stream, flush_l2, seed, hbm):
                            "gather_quantise": rate(b_g, ms_g, hbm), "decode_us": round(ms_d * 1e3, 2),
                            "decode_bytes": b_d, "decode": rate(b_d, ms_d, hbm)}
     del kb, vb, kq, vq, d7
+
+    # -- xKV: factorise the keys of a window of W = 4 layers (S = 32768, r = 64, bf16 basis, 8 iteration steps),
+    #    then rebuild 2048 selected rows per head of one layer (selective) and all S rows (dense)
+    S8, W8, r8, it8 = 32768, 4, 64, 8
+    F8 = W8 * d
+    keys8 = [torch.randn((S8, n_kv, d), device=dev).to(torch.bfloat16) for _ in range(W8)]
+    gen8 = torch.Generator(device=dev)
+    gen8.manual_seed(seed + 8)
+    v08 = torch.randn((n_kv, F8, r8), generator=gen8, device=dev)
+    basis8 = torch.empty((n_kv, S8, r8), dtype=torch.bfloat16, device=dev)
+    blocks8 = torch.empty((n_kv, r8, F8), dtype=torch.float32, device=dev)
+    ws8 = torch.empty(kvc.kvc_xkv_workspace_size(S8, n_kv, d, W8, r8), dtype=torch.uint8, device=dev)
+    ms_f, _, nl_f = time_graph([lambda: kvc.kvc_xkv_factorize(keys8, r8, it8, v08, basis8, blocks8, ws8)], flush_l2,
+                               stream, steps)
+    gram_flops = 2 * S8 * F8 * F8 * n_kv
+    b_f = 2 * W8 * S8 * n_kv * d * 2 + n_kv * S8 * r8 * 2         # keys read by the Gram and the projection, A written
+    res = {"factorize_us": round(ms_f * 1e3, 2), "factorize_kernels": nl_f, "iters": it8,
+           "gram_tflops_equiv": round(gram_flops / (ms_f * 1e-3) / 1e12, 1), "factorize_bytes": b_f,
+           "factorize": rate(b_f, ms_f, hbm)}
+    for n_sel, tag in ((2048, "selective_2048"), (S8, "dense")):
+        idx8 = torch.randint(0, S8, (n_kv, n_sel), dtype=torch.int32, device=dev)
+        out8 = torch.empty((n_sel, n_kv, d), dtype=torch.bfloat16, device=dev)
+        ms_r, _, nl_r = time_graph([lambda: kvc.kvc_xkv_reconstruct(W8, 1, basis8, blocks8, idx8, out8)], flush_l2,
+                                   stream, steps)
+        b_r = n_sel * n_kv * (r8 * 2 + d * 2 + 4) + n_kv * r8 * d * 4
+        res[f"rebuild_{tag}_us"] = round(ms_r * 1e3, 2)
+        res[f"rebuild_{tag}_bytes"] = b_r
+        res[f"rebuild_{tag}"] = rate(b_r, ms_r, hbm)
+        res[f"rebuild_{tag}_gflops"] = round(2 * n_sel * n_kv * r8 * d / (ms_r * 1e-3) / 1e9, 1)
+        del idx8, out8
+    out[f"xkv_S{S8}_W{W8}_r{r8}"] = res
+    del keys8, v08, basis8, blocks8, ws8
     torch.cuda.empty_cache()
     return out
 

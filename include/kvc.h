@@ -356,6 +356,56 @@ kvc_status kvc_freekv_step(int batch, const int32_t *seqlens_host, const int32_t
                            const void *v, int32_t *idx, void *k_c, void *v_c, int32_t *reselected, float *out,
                            void *ws, size_t ws_bytes, kvc_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * xKV cross-layer factorisation and selective reconstruction.  Source: "xKV -
+ * Compression de Cache KV Inter-couche par Extraction de Vecteurs Singuliers
+ * Alignes" (gist.science 2503.18893), technical summary section 2.2
+ * ("Factorisation Inter-couche": the caches of a window of W consecutive
+ * layers are concatenated along the features, a rank-r SVD of the result
+ * gives a token basis shared by the window and one reconstruction matrix per
+ * layer) and section 2.3 ("Reconstruction Selective": only the rows of the
+ * chosen tokens are rebuilt, from the shared basis and the layer's matrix).
+ *
+ * One sequence of S tokens; the factorisation is per KV head h:
+ *   X_h = [K_0[:, h] | K_1[:, h] | ... | K_{W-1}[:, h]]   (S x F, F = W d_h)
+ *   Vt_h (r x F) spans the top-r right singular subspace of X_h (orthonormal
+ *     rows), A_h = X_h Vt_h^T (S x r), so A_h Vt_h is the rank-r truncated SVD
+ *     of X_h; layer l's reconstruction matrix is Vt_h[:, l d_h : (l+1) d_h].
+ * The subspace is computed by `iters` steps of subspace iteration on the
+ * Gram matrix X_h^T X_h (float32, bf16 products) from the start basis v0,
+ * each step re-orthonormalised by Cholesky-QR in float64.  Its distance to
+ * the exact singular subspace shrinks like (s_{r+1} / s_r)^(2 iters) (s: the
+ * singular values of X_h) down to float32 resolution; where s_r = s_{r+1} the
+ * subspace is not unique and any converged one is valid.  A_h and Vt_h are
+ * unique only up to a rotation of the r basis vectors; A_h Vt_h is unique.
+ *
+ * kvc_xkv_factorize: bf16 only.  d_h in {64, 128}; 1 <= W <= 8; W d_h <= 512;
+ * r in {16, 32, 64}, r <= min(S, W d_h); 1 <= iters <= 1000.
+ *   k_layers: host array of W device pointers, each bf16 [S, n_kv, d_h] (the
+ *     keys of the window's layers; values are factorised the same way by a
+ *     second call).
+ *   v0: float32 [n_kv, W d_h, r] start basis (e.g. Gaussian; its columns must
+ *     not be orthogonal to the top-r subspace).
+ *   basis_dt: KVC_F32 or KVC_BF16 (round to nearest even) for A.
+ *   basis: [n_kv, S, r] of basis_dt (A_h);  blocks: float32 [n_kv, r, W d_h]
+ *     (Vt_h).  ws: kvc_xkv_workspace_size() bytes; no zeroing needed.
+ *
+ * kvc_xkv_reconstruct: rows idx[h][t] (t < n_sel) of layer `layer`:
+ *   out[t][h][:] = bf16_rn( A_h[idx[h][t]] Vt_h[:, layer d_h : (layer+1) d_h] )
+ *   idx: int32 [n_kv, n_sel] (e.g. a kvc_select_topk segment); an index
+ *   outside [0, S) yields a zero row.  out: bf16 [n_sel, n_kv, d_h], the
+ *   layout of a compact cache, ready for kvc_gqa_decode_attn.  Shapes and
+ *   basis_dt as given to kvc_xkv_factorize.
+ * Both calls are asynchronous on `stream`; errors as for every entry point.
+ * ------------------------------------------------------------------------ */
+size_t kvc_xkv_workspace_size(int S, int n_kv, int d_h, int W, int r);
+kvc_status kvc_xkv_factorize(int S, int n_kv, int d_h, int W, int r, int iters, const void *const *k_layers,
+                             const float *v0, kvc_dtype basis_dt, void *basis, float *blocks, void *ws,
+                             size_t ws_bytes, kvc_stream_t stream);
+kvc_status kvc_xkv_reconstruct(int S, int n_kv, int d_h, int W, int r, int layer, int n_sel, kvc_dtype basis_dt,
+                               const void *basis, const float *blocks, const int32_t *idx, void *out,
+                               kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

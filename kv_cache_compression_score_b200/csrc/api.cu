@@ -707,3 +707,105 @@ extern "C" kvc_status kvc_tsp_select_gather_static(kvc_dtype dt, int S, int n_ro
   if (e != cudaSuccess) return cuda_fail(e, "hidden gather kernel");
   return KVC_OK;
 }
+
+// ----------------------------------------------------------------- xKV
+namespace {
+struct XkvPlan {
+  int F = 0;
+  size_t off_gram = 0, off_y = 0, off_va = 0, off_vb = 0, off_c = 0, off_m = 0, bytes = 0;
+};
+
+kvc_status check_xkv_shape(int S, int n_kv, int d_h, int W, int r) {
+  if (S < 1 || n_kv < 1) return fail(KVC_ERR_INVALID_ARG, "S and n_kv must be >= 1 (S=%d, n_kv=%d)", S, n_kv);
+  if (n_kv > 65535) return fail(KVC_ERR_UNSUPPORTED, "n_kv must be <= 65535");
+  if (d_h != 64 && d_h != 128) return fail(KVC_ERR_UNSUPPORTED, "d_h must be 64 or 128 (got %d)", d_h);
+  if (W < 1 || W > kvc::kXkvMaxW) return fail(KVC_ERR_UNSUPPORTED, "W must be in [1, %d] (got %d)", kvc::kXkvMaxW, W);
+  const int F = W * d_h;
+  if (F > 512) return fail(KVC_ERR_UNSUPPORTED, "W * d_h must be <= 512 (got %d)", F);
+  if (r != 16 && r != 32 && r != 64) return fail(KVC_ERR_UNSUPPORTED, "r must be 16, 32 or 64 (got %d)", r);
+  if (r > S || r > F) return fail(KVC_ERR_INVALID_ARG, "r (%d) must be <= min(S, W * d_h) = %d", r, std::min(S, F));
+  return KVC_OK;
+}
+
+kvc_status plan_xkv(int S, int n_kv, int d_h, int W, int r, XkvPlan *pl) {
+  kvc_status s = check_xkv_shape(S, n_kv, d_h, W, r);
+  if (s != KVC_OK) return s;
+  pl->F = W * d_h;
+  const size_t nk = (size_t)n_kv;
+  pl->off_gram = kErrWordBytes;
+  pl->off_y = round_up(pl->off_gram + nk * pl->F * pl->F * sizeof(float), 256);
+  pl->off_va = round_up(pl->off_y + nk * pl->F * r * sizeof(float), 256);
+  pl->off_vb = round_up(pl->off_va + nk * pl->F * r * sizeof(float), 256);
+  pl->off_c = round_up(pl->off_vb + nk * pl->F * r * sizeof(float), 256);
+  pl->off_m = round_up(pl->off_c + nk * r * r * sizeof(double), 256);
+  pl->bytes = round_up(pl->off_m + nk * r * r * sizeof(double), 256);
+  return KVC_OK;
+}
+}  // namespace
+
+extern "C" size_t kvc_xkv_workspace_size(int S, int n_kv, int d_h, int W, int r) {
+  XkvPlan pl;
+  return plan_xkv(S, n_kv, d_h, W, r, &pl) == KVC_OK ? pl.bytes : 0;
+}
+
+extern "C" kvc_status kvc_xkv_factorize(int S, int n_kv, int d_h, int W, int r, int iters,
+                                        const void *const *k_layers, const float *v0, kvc_dtype basis_dt,
+                                        void *basis, float *blocks, void *ws, size_t ws_bytes,
+                                        kvc_stream_t stream) {
+  XkvPlan pl;
+  kvc_status s = plan_xkv(S, n_kv, d_h, W, r, &pl);
+  if (s != KVC_OK) return s;
+  if (iters < 1 || iters > 1000) return fail(KVC_ERR_INVALID_ARG, "iters must be in [1, 1000] (got %d)", iters);
+  if (basis_dt != KVC_F32 && basis_dt != KVC_BF16)
+    return fail(KVC_ERR_UNSUPPORTED, "basis dtype %d not supported", (int)basis_dt);
+  if (!k_layers) return fail(KVC_ERR_INVALID_ARG, "k_layers is NULL");
+  for (int l = 0; l < W; ++l)
+    if (!aligned16(k_layers[l])) return fail(KVC_ERR_INVALID_ARG, "k_layers[%d] must be non-NULL and 16-byte aligned", l);
+  if (!aligned16(v0) || !aligned16(basis) || !aligned16(blocks))
+    return fail(KVC_ERR_INVALID_ARG, "v0, basis and blocks must be non-NULL and 16-byte aligned");
+  if (!aligned16(ws)) return fail(KVC_ERR_WORKSPACE, "ws must be non-NULL and 16-byte aligned");
+  if (ws_bytes < pl.bytes)
+    return fail(KVC_ERR_WORKSPACE, "workspace of %zu bytes is below the %zu required", ws_bytes, pl.bytes);
+  char *w = static_cast<char *>(ws);
+  kvc::XkvArgs a = {};
+  a.S = S; a.n_kv = n_kv; a.d_h = d_h; a.W = W; a.r = r; a.iters = iters;
+  for (int l = 0; l < W; ++l) a.k_layers[l] = k_layers[l];
+  a.v0 = v0;
+  a.gram = reinterpret_cast<float *>(w + pl.off_gram);
+  a.y = reinterpret_cast<float *>(w + pl.off_y);
+  a.v_a = reinterpret_cast<float *>(w + pl.off_va);
+  a.v_b = reinterpret_cast<float *>(w + pl.off_vb);
+  a.c = reinterpret_cast<double *>(w + pl.off_c);
+  a.m = reinterpret_cast<double *>(w + pl.off_m);
+  a.blocks = blocks;
+  a.basis = basis;
+  a.basis_bf16 = basis_dt == KVC_BF16;
+  cudaError_t e = kvc::xkv_factorize(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "xKV factorisation kernels");
+  return KVC_OK;
+}
+
+extern "C" kvc_status kvc_xkv_reconstruct(int S, int n_kv, int d_h, int W, int r, int layer, int n_sel,
+                                          kvc_dtype basis_dt, const void *basis, const float *blocks,
+                                          const int32_t *idx, void *out, kvc_stream_t stream) {
+  kvc_status s = check_xkv_shape(S, n_kv, d_h, W, r);
+  if (s != KVC_OK) return s;
+  if (layer < 0 || layer >= W) return fail(KVC_ERR_INVALID_ARG, "layer must be in [0, W) (got %d)", layer);
+  if (n_sel < 0) return fail(KVC_ERR_INVALID_ARG, "n_sel must be >= 0");
+  if (n_sel > INT32_MAX - 64) return fail(KVC_ERR_UNSUPPORTED, "n_sel too large");
+  if (basis_dt != KVC_F32 && basis_dt != KVC_BF16)
+    return fail(KVC_ERR_UNSUPPORTED, "basis dtype %d not supported", (int)basis_dt);
+  if (!aligned16(basis) || !aligned16(blocks) || !aligned16(idx) || !aligned16(out))
+    return fail(KVC_ERR_INVALID_ARG, "basis, blocks, idx and out must be non-NULL and 16-byte aligned");
+  if (n_sel == 0) return KVC_OK;
+  kvc::XkvArgs a = {};
+  a.S = S; a.n_kv = n_kv; a.d_h = d_h; a.W = W; a.r = r; a.layer = layer; a.n_sel = n_sel;
+  a.basis = const_cast<void *>(basis);
+  a.blocks = const_cast<float *>(blocks);
+  a.basis_bf16 = basis_dt == KVC_BF16;
+  a.idx = idx;
+  a.out = out;
+  cudaError_t e = kvc::xkv_reconstruct(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "xKV reconstruction kernel");
+  return KVC_OK;
+}

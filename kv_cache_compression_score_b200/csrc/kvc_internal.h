@@ -112,6 +112,26 @@ cudaError_t gqa_decode(const DecodeArgs &a, cudaStream_t st);
 cudaError_t gqa_decode_tc(const DecodeArgs &a, cudaStream_t st);   // bf16 / int8 caches, tensor cores
 int decode_slots(int max_kv_len);
 
+// xKV cross-layer factorisation (xkv.cu)
+constexpr int kXkvMaxW = 8;
+struct XkvArgs {
+  int S, n_kv, d_h, W, r, iters;
+  const void *k_layers[kXkvMaxW];   // bf16 key caches [S, n_kv, d_h] of the window's layers
+  const float *v0;                  // [n_kv, W d_h, r] start basis
+  float *gram, *y, *v_a, *v_b;      // workspace
+  double *c, *m;                    // workspace
+  float *blocks;                    // Vt [n_kv, r, W d_h]
+  void *basis;                      // A [n_kv, S, r] float32 or bf16
+  bool basis_bf16;
+  // reconstruction
+  int layer, n_sel;
+  const int32_t *idx;               // [n_kv, n_sel]
+  void *out;                        // bf16 [n_sel, n_kv, d_h]
+};
+cudaError_t xkv_factorize(const XkvArgs &a, cudaStream_t st);
+cudaError_t xkv_reconstruct(const XkvArgs &a, cudaStream_t st);
+int xkv_gram_split_tokens(int S, int n_kv, int F);
+
 }  // namespace kvc
 
 namespace kvc {

@@ -53,6 +53,11 @@ SIGNATURES = {
     "kvc_freekv_workspace_size": (_c_sz, [_c_int, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "kvc_freekv_step": (_c_int, [_c_int, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_f,
                                  _c_f, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "kvc_xkv_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "kvc_xkv_factorize": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p, _c_int, _c_p, _c_p,
+                                   _c_p, _c_sz, _c_p]),
+    "kvc_xkv_reconstruct": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p,
+                                     _c_p, _c_p, _c_p]),
     "kvc_gqa_decode_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "kvc_gqa_decode_attn": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_i64, _c_p,
                                      _c_p, _c_int, _c_p, _c_p, _c_sz, _c_p]),
@@ -260,3 +265,27 @@ def kvc_freekv_step(seqlens, cu_seqlens, cu_budget, n_h: int, w: int, pool_k: in
                                  pool_k, budget, tau, scale, _dptr(q_cur), _dptr(q_prev), _dptr(k), _dptr(v),
                                  _dptr(idx), _dptr(k_c), _dptr(v_c), _dptr(reselected), _dptr(out), _dptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_xkv_workspace_size(S: int, n_kv: int, d_h: int, W: int, r: int) -> int:
+    return int(lib().kvc_xkv_workspace_size(S, n_kv, d_h, W, r))
+
+
+def kvc_xkv_factorize(k_layers, r: int, iters: int, v0, basis, blocks, ws, stream=None) -> None:
+    """xKV factorisation of the keys of W layers (list of bf16 [S, n_kv, d_h]
+    tensors): writes basis (A, [n_kv, S, r], float32 or bf16) and blocks (Vt,
+    float32 [n_kv, r, W d_h])."""
+    S, n_kv, d_h = k_layers[0].shape
+    ptrs = (ctypes.c_void_p * len(k_layers))(*[t.data_ptr() for t in k_layers])
+    _check(lib().kvc_xkv_factorize(S, n_kv, d_h, len(k_layers), r, iters, ptrs, _dptr(v0), dtype_code(basis),
+                                   _dptr(basis), _dptr(blocks), _dptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)))
+
+
+def kvc_xkv_reconstruct(W: int, layer: int, basis, blocks, idx, out, stream=None) -> None:
+    """Rows idx ([n_kv, n_sel] int32) of layer `layer` into out (bf16 [n_sel, n_kv, d_h])."""
+    n_kv, S, r = basis.shape
+    n_sel = idx.shape[1]
+    d_h = out.shape[2]
+    _check(lib().kvc_xkv_reconstruct(S, n_kv, d_h, W, r, layer, n_sel, dtype_code(basis), _dptr(basis),
+                                     _dptr(blocks), _dptr(idx), _dptr(out), _stream(stream)))

@@ -27,7 +27,7 @@ MASK64 = np.uint64(0xFFFFFFFFFFFFFFFF)
 GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
 
 # Tensor ids: one independent stream per (seed, id, sequence).
-T_QWIN, T_K, T_V, T_QDEC, T_HIDDEN, T_BOOST_DIR, T_BOOST_POS, T_LENGTHS, T_SCORES, T_DRIFT = range(1, 11)
+T_QWIN, T_K, T_V, T_QDEC, T_HIDDEN, T_BOOST_DIR, T_BOOST_POS, T_LENGTHS, T_SCORES, T_DRIFT, T_XKV = range(1, 12)
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -202,3 +202,31 @@ def drifted_queries(seed: int, q_prev_bits: np.ndarray, dtype: str, lo: float = 
     sig = np.repeat(sig.reshape(batch, n_h // group), group, axis=1).reshape(batch, n_h, 1)
     noise = normal_f64(stream_key(seed, T_DRIFT, 1), batch * n_h * d).reshape(batch, n_h, d)
     return round_to(prev + sig * noise, dtype)
+
+
+def cross_layer_keys(seed: int, S: int, n_kv: int, d_h: int, W: int, rank: int, noise: float = 0.05,
+                     dtype: str = "bf16") -> list:
+    """Keys of W layers, [S, n_kv, d_h] each, whose per-head concatenation
+    [K_1[:, h] | ... | K_W[:, h]] is a rank-`rank` matrix plus noise: a token
+    factor Z_h ([S, rank], N(0,1), column c scaled by 2^(-2c/rank)) shared by
+    the W layers, times per-layer loadings ([rank, d_h], N(0,1) / sqrt(rank)),
+    plus noise * N(0,1) per element.  The shared token factor stands for the
+    aligned dominant singular vectors across layers that the xKV page reports;
+    the scaled columns give a decaying spectrum with a gap after `rank`."""
+    F = W * d_h
+    out = np.zeros((W, S, n_kv, d_h))
+    col = 2.0 ** (-2.0 * np.arange(rank) / rank)
+    for h in range(n_kv):
+        Z = normal_f64(stream_key(seed, T_XKV, 3 * h), S * rank).reshape(S, rank) * col
+        B = normal_f64(stream_key(seed, T_XKV, 3 * h + 1), rank * F).reshape(rank, F) / np.sqrt(rank)
+        E = normal_f64(stream_key(seed, T_XKV, 3 * h + 2), S * F).reshape(S, F) * noise
+        X = Z @ B + E
+        for l in range(W):
+            out[l, :, h, :] = X[:, l * d_h:(l + 1) * d_h]
+    return [round_to(out[l], dtype) for l in range(W)]
+
+
+def start_basis(seed: int, n_kv: int, F: int, r: int) -> np.ndarray:
+    """Gaussian start basis [n_kv, F, r] (float32) for subspace iteration."""
+    key = stream_key(seed, T_XKV, 0xFFFF)
+    return normal_f64(key, n_kv * F * r).reshape(n_kv, F, r).astype(np.float32)

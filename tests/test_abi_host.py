@@ -137,6 +137,39 @@ def test_select_gather_decode_tsp_reject_before_launch(L):
                                    None) == UNSUPPORTED
 
 
+def test_xkv_rejects_before_launch(L):
+    ptrs = (ctypes.c_void_p * 8)(*([P16.value] * 8))
+    ws_ok = kvc.kvc_xkv_workspace_size(256, 2, 128, 4, 64)
+    assert ws_ok >= 2 * 512 * 512 * 4                    # holds the Gram matrices
+    assert kvc.kvc_xkv_workspace_size(256, 2, 128, 5, 64) == 0     # W d_h = 640 > 512
+    assert kvc.kvc_xkv_workspace_size(256, 2, 96, 2, 16) == 0      # d_h unsupported
+    assert kvc.kvc_xkv_workspace_size(40, 2, 128, 2, 64) == 0      # r > S
+
+    def fac(S=256, n_kv=2, d=128, W=4, r=64, iters=8, kl=ptrs, v0=P16, bdt=kvc.KVC_BF16, basis=P16, ws_b=ws_ok):
+        return L.kvc_xkv_factorize(S, n_kv, d, W, r, iters, kl, v0, bdt, basis, P16, P16, ws_b, None)
+
+    assert fac(r=48) == UNSUPPORTED
+    assert fac(W=9) == UNSUPPORTED
+    assert fac(iters=0) == INVALID
+    assert fac(bdt=7) == UNSUPPORTED
+    assert fac(kl=None) == INVALID
+    assert fac(kl=(ctypes.c_void_p * 8)(*([P8.value] * 8))) == INVALID
+    assert fac(v0=None) == INVALID
+    assert fac(basis=P8) == INVALID
+    assert fac(ws_b=64) == WORKSPACE
+    assert fac(S=32, r=64) == INVALID
+
+    def rec(layer=0, n_sel=10, r=64, idx=P16):
+        return L.kvc_xkv_reconstruct(256, 2, 128, 4, r, layer, n_sel, kvc.KVC_BF16, P16, P16, idx, P16, None)
+
+    assert rec(layer=4) == INVALID
+    assert rec(layer=-1) == INVALID
+    assert rec(n_sel=-1) == INVALID
+    assert rec(r=8) == UNSUPPORTED
+    assert rec(idx=P8) == INVALID
+    assert rec(n_sel=0) == 0                               # nothing to do, nothing launched
+
+
 def test_check_workspace_and_launch_count_need_no_gpu_to_validate(L):
     """kvc_check_workspace rejects a NULL workspace before any CUDA call; the
     launch counter is readable without a device."""
