@@ -411,10 +411,13 @@ def rate(bytes_, ms, hbm):
     return {"gbs": round(gbs, 1), "frac_of_measured_peak": round(gbs / hbm, 3), "frac_of_8000": round(gbs / 8000, 3)}
 
 
-def run_workloads(args, dev, stream, flush_l2, seed, hbm):
-    """Every workload of the benchmark set besides the headline layer, each
-    through the C ABI in one CUDA graph, with algorithmic bytes and the
-    fraction of the measured HBM peak."""
+WORKLOAD_NAMES = ("pr1", "s131072", "fastkv", "ragged", "freekv", "q8", "xkv")
+
+
+def run_workloads(args, dev, stream, flush_l2, seed, hbm, only=None):
+    """Every workload of the benchmark set besides the headline layer (or the
+    one named by `only`), each through the C ABI in one CUDA graph, with
+    algorithmic bytes and the fraction of the measured HBM peak."""
     import torch
     from kv_cache_compression_score_b200 import kvc, synth
     from kv_cache_compression_score_b200.runner import Compressor, Decoder, FreeKvStep, TspSelector, to_device
@@ -423,193 +426,201 @@ def run_workloads(args, dev, stream, flush_l2, seed, hbm):
     n_h, n_kv, d, w, pk = 32, 8, 128, 32, 7
     row = n_kv * d * 2                                   # bytes of one bf16 cache row (all KV heads)
 
-    # -- PR1: one fp32 layer, n_h 4, n_kv 2, d_h 64, S 2048, B 256, one decode query
-    bt = synth.packed_batch(1001, [2048], 4, 2, 64, 32, "f32")
-    q1, k1, v1 = (to_device(bt[x], "f32", dev) for x in ("q_win", "k", "v"))
-    c1 = Compressor("f32", [2048], 4, 2, 64, 32, pk, 256, device=dev, keep_raw=False)
-    d1 = Decoder(1, 4, 2, 64, 256, device=dev)
-    qd1 = to_device(synth.decode_queries(1009, 1, 4, 64, "f32"), "f32", dev)
-    z1 = torch.zeros(1, dtype=torch.int64, device=dev)
-    l1 = torch.full((1,), 256, dtype=torch.int32, device=dev)
-    ms, mn, nl = time_graph([lambda: c1.compress(q1, k1, v1), lambda: d1.run(qd1, c1.buf.k_c, c1.buf.v_c, z1, l1)],
-                            flush_l2, stream, steps)
-    b_ssg, b_dec = 2048 * 2 * 64 * 4 + 2 * 2 * 256 * 2 * 64 * 4, 2 * 256 * 2 * 64 * 4
-    out["pr1_f32_S2048_B256"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
-                                 "ktok_s": round(2048 / (ms * 1e-3) / 1e3, 1), "bytes": b_ssg + b_dec,
-                                 **rate(b_ssg + b_dec, ms, hbm), "note": "latency-bound (1.8 MB)"}
-    del c1, d1, q1, k1, v1
+    if only in (None, "pr1"):
+        # -- PR1: one fp32 layer, n_h 4, n_kv 2, d_h 64, S 2048, B 256, one decode query
+        bt = synth.packed_batch(1001, [2048], 4, 2, 64, 32, "f32")
+        q1, k1, v1 = (to_device(bt[x], "f32", dev) for x in ("q_win", "k", "v"))
+        c1 = Compressor("f32", [2048], 4, 2, 64, 32, pk, 256, device=dev, keep_raw=False)
+        d1 = Decoder(1, 4, 2, 64, 256, device=dev)
+        qd1 = to_device(synth.decode_queries(1009, 1, 4, 64, "f32"), "f32", dev)
+        z1 = torch.zeros(1, dtype=torch.int64, device=dev)
+        l1 = torch.full((1,), 256, dtype=torch.int32, device=dev)
+        ms, mn, nl = time_graph([lambda: c1.compress(q1, k1, v1), lambda: d1.run(qd1, c1.buf.k_c, c1.buf.v_c, z1, l1)],
+                                flush_l2, stream, steps)
+        b_ssg, b_dec = 2048 * 2 * 64 * 4 + 2 * 2 * 256 * 2 * 64 * 4, 2 * 256 * 2 * 64 * 4
+        out["pr1_f32_S2048_B256"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
+                                     "ktok_s": round(2048 / (ms * 1e-3) / 1e3, 1), "bytes": b_ssg + b_dec,
+                                     **rate(b_ssg + b_dec, ms, hbm), "note": "latency-bound (1.8 MB)"}
+        del c1, d1, q1, k1, v1
 
-    # -- S = 131072: B = 4096, B = S (identity), decode at batch 8, full-cache decode
-    S3 = 131072
-    q3, k3, v3 = device_inputs(seed + 3, [S3], n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
-    for B3, name in ((4096, "llama8b_S131072_B4096"), (S3, "llama8b_S131072_B=S")):
-        c3 = Compressor("bf16", [S3], n_h, n_kv, d, w, pk, B3, device=dev, keep_raw=False)
-        ms, mn, nl = time_graph([lambda: c3.compress(q3, k3, v3)], flush_l2, stream, steps)
-        b = S3 * row + 2 * 2 * B3 * row
-        out[name] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
-                     "ktok_s": round(S3 / (ms * 1e-3) / 1e3, 1), "bytes": b, **rate(b, ms, hbm)}
-        if B3 == 4096:
-            # decode at batch 8 over compact caches of 4096 rows (cache 0 from this step)
-            kc8 = torch.randn((8 * B3, n_kv, d), device=dev).to(torch.bfloat16)
-            vc8 = torch.randn_like(kc8)
-            qd8 = torch.randn((8, n_h, d), device=dev).to(torch.bfloat16)
-            off8 = torch.arange(8, dtype=torch.int64, device=dev) * B3
-            ln8 = torch.full((8,), B3, dtype=torch.int32, device=dev)
-            dd = Decoder(8, n_h, n_kv, d, B3, device=dev)
-            ms, mn, nl = time_graph([lambda: dd.run(qd8, kc8, vc8, off8, ln8)], flush_l2, stream, steps)
-            b = 8 * B3 * row * 2
-            out["decode_b8_B4096"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
-                                      "bytes": b, **rate(b, ms, hbm)}
-            del kc8, vc8, dd
-        del c3
-    # full-cache decode: 8 independent caches of 131072 rows (4 GiB of K and V)
-    kf = torch.empty((8 * S3, n_kv, d), dtype=torch.bfloat16, device=dev)
-    vf = torch.empty_like(kf)
-    for i in range(8):
-        kf[i * S3:(i + 1) * S3].copy_(k3)
-        vf[i * S3:(i + 1) * S3].copy_(v3)
-    qd8 = torch.randn((8, n_h, d), device=dev).to(torch.bfloat16)
-    off8 = torch.arange(8, dtype=torch.int64, device=dev) * S3
-    ln8 = torch.full((8,), S3, dtype=torch.int32, device=dev)
-    dd = Decoder(8, n_h, n_kv, d, S3, device=dev)
-    ms, mn, nl = time_graph([lambda: dd.run(qd8, kf, vf, off8, ln8)], flush_l2, stream, steps)
-    b = 8 * S3 * row * 2
-    out["full_cache_decode_b8_S131072"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
-                                           "bytes": b, **rate(b, ms, hbm)}
-    del kf, vf, dd, q3, k3, v3
+    if only in (None, "s131072"):
+        # -- S = 131072: B = 4096, B = S (identity), decode at batch 8, full-cache decode
+        S3 = 131072
+        q3, k3, v3 = device_inputs(seed + 3, [S3], n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
+        for B3, name in ((4096, "llama8b_S131072_B4096"), (S3, "llama8b_S131072_B=S")):
+            c3 = Compressor("bf16", [S3], n_h, n_kv, d, w, pk, B3, device=dev, keep_raw=False)
+            ms, mn, nl = time_graph([lambda: c3.compress(q3, k3, v3)], flush_l2, stream, steps)
+            b = S3 * row + 2 * 2 * B3 * row
+            out[name] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
+                         "ktok_s": round(S3 / (ms * 1e-3) / 1e3, 1), "bytes": b, **rate(b, ms, hbm)}
+            if B3 == 4096:
+                # decode at batch 8 over compact caches of 4096 rows (cache 0 from this step)
+                kc8 = torch.randn((8 * B3, n_kv, d), device=dev).to(torch.bfloat16)
+                vc8 = torch.randn_like(kc8)
+                qd8 = torch.randn((8, n_h, d), device=dev).to(torch.bfloat16)
+                off8 = torch.arange(8, dtype=torch.int64, device=dev) * B3
+                ln8 = torch.full((8,), B3, dtype=torch.int32, device=dev)
+                dd = Decoder(8, n_h, n_kv, d, B3, device=dev)
+                ms, mn, nl = time_graph([lambda: dd.run(qd8, kc8, vc8, off8, ln8)], flush_l2, stream, steps)
+                b = 8 * B3 * row * 2
+                out["decode_b8_B4096"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
+                                          "bytes": b, **rate(b, ms, hbm)}
+                del kc8, vc8, dd
+            del c3
+        # full-cache decode: 8 independent caches of 131072 rows (4 GiB of K and V)
+        kf = torch.empty((8 * S3, n_kv, d), dtype=torch.bfloat16, device=dev)
+        vf = torch.empty_like(kf)
+        for i in range(8):
+            kf[i * S3:(i + 1) * S3].copy_(k3)
+            vf[i * S3:(i + 1) * S3].copy_(v3)
+        qd8 = torch.randn((8, n_h, d), device=dev).to(torch.bfloat16)
+        off8 = torch.arange(8, dtype=torch.int64, device=dev) * S3
+        ln8 = torch.full((8,), S3, dtype=torch.int32, device=dev)
+        dd = Decoder(8, n_h, n_kv, d, S3, device=dev)
+        ms, mn, nl = time_graph([lambda: dd.run(qd8, kf, vf, off8, ln8)], flush_l2, stream, steps)
+        b = 8 * S3 * row * 2
+        out["full_cache_decode_b8_S131072"] = {"us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl,
+                                               "bytes": b, **rate(b, ms, hbm)}
+        del kf, vf, dd, q3, k3, v3
 
-    # -- FastKV: 32 layers, TSP at layer 15 (k_tsp = floor(0.2 S) + w), hidden [S, 4096]
-    S4, L4 = 32768, 32
-    k_tsp, b_avg = (S4 * 2) // 10, S4 // 10
-    S4n = k_tsp + w
-    layers = []
-    for layer in range(L4):
-        length = S4 if layer <= 15 else S4n
-        layers.append(device_inputs(seed + 100 + layer, [length], n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev))
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(seed + 200)
-    hidden = torch.randn((S4, 4096), generator=gen, device=dev).to(torch.bfloat16)
-    for sched in ("uniform", "pyramid"):
-        budgets = [b_avg] * L4 if sched == "uniform" else [int(x) for x in kvc.kvc_pyramid_budgets(L4, b_avg, 1024)]
-        comps = [Compressor("bf16", [S4 if l <= 15 else S4n], n_h, n_kv, d, w, pk, budgets[l], device=dev,
-                            keep_raw=(l == 15)) for l in range(L4)]
-        tsp = TspSelector(S4, w, pk, k_tsp, 4096, "bf16", device=dev)
-        fns = [(lambda c=c, x=x: c.compress(*x)) for c, x in zip(comps, layers)]
-        fns.insert(16, lambda: tsp.run(comps[15].buf.scores_raw, hidden))
-        ms, mn, nl = time_graph(fns, flush_l2, stream, max(3, steps // 2))
-        b = sum((S4 if l <= 15 else S4n) * row + 2 * 2 * min(budgets[l], S4 if l <= 15 else S4n) * row
-                for l in range(L4)) + 2 * (k_tsp + w) * 4096 * 2
-        out[f"fastkv_32_layer_chain_{sched}"] = {
-            "us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl, "bytes": b, **rate(b, ms, hbm),
-            "budgets": [budgets[0], budgets[15], budgets[31]] if sched == "pyramid" else b_avg}
-        del comps, tsp
-    del layers, hidden
+    if only in (None, "fastkv"):
+        # -- FastKV: 32 layers, TSP at layer 15 (k_tsp = floor(0.2 S) + w), hidden [S, 4096]
+        S4, L4 = 32768, 32
+        k_tsp, b_avg = (S4 * 2) // 10, S4 // 10
+        S4n = k_tsp + w
+        layers = []
+        for layer in range(L4):
+            length = S4 if layer <= 15 else S4n
+            layers.append(device_inputs(seed + 100 + layer, [length], n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev))
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed + 200)
+        hidden = torch.randn((S4, 4096), generator=gen, device=dev).to(torch.bfloat16)
+        for sched in ("uniform", "pyramid"):
+            budgets = [b_avg] * L4 if sched == "uniform" else [int(x) for x in kvc.kvc_pyramid_budgets(L4, b_avg, 1024)]
+            comps = [Compressor("bf16", [S4 if l <= 15 else S4n], n_h, n_kv, d, w, pk, budgets[l], device=dev,
+                                keep_raw=(l == 15)) for l in range(L4)]
+            tsp = TspSelector(S4, w, pk, k_tsp, 4096, "bf16", device=dev)
+            fns = [(lambda c=c, x=x: c.compress(*x)) for c, x in zip(comps, layers)]
+            fns.insert(16, lambda: tsp.run(comps[15].buf.scores_raw, hidden))
+            ms, mn, nl = time_graph(fns, flush_l2, stream, max(3, steps // 2))
+            b = sum((S4 if l <= 15 else S4n) * row + 2 * 2 * min(budgets[l], S4 if l <= 15 else S4n) * row
+                    for l in range(L4)) + 2 * (k_tsp + w) * 4096 * 2
+            out[f"fastkv_32_layer_chain_{sched}"] = {
+                "us": round(ms * 1e3, 2), "min_us": round(mn * 1e3, 2), "kernels": nl, "bytes": b, **rate(b, ms, hbm),
+                "budgets": [budgets[0], budgets[15], budgets[31]] if sched == "pyramid" else b_avg}
+            del comps, tsp
+        del layers, hidden
 
-    # -- ragged batch: 16 lengths uniform on [4096, 65536], B = min(1024, len), then decode over the 16 caches
-    lens5 = [int(x) for x in synth.ragged_lengths(1005, 16, 4096, 65536)]
-    q5, k5, v5 = device_inputs(seed + 5, lens5, n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
-    c5 = Compressor("bf16", lens5, n_h, n_kv, d, w, pk, 1024, device=dev, keep_raw=False)
-    cb5 = c5.buf.cu_budget_host
-    off5 = torch.tensor(cb5[:-1], dtype=torch.int64, device=dev)
-    ln5 = torch.tensor(np.diff(cb5), dtype=torch.int32, device=dev)
-    qd5 = torch.randn((16, n_h, d), device=dev).to(torch.bfloat16)
-    d5 = Decoder(16, n_h, n_kv, d, 1024, device=dev)
-    ms_c, mn_c, nl_c = time_graph([lambda: c5.compress(q5, k5, v5)], flush_l2, stream, steps)
-    ms_d, mn_d, nl_d = time_graph([lambda: d5.run(qd5, c5.buf.k_c, c5.buf.v_c, off5, ln5)], flush_l2, stream, steps)
-    b_c = sum(lens5) * row + 2 * 2 * 16 * 1024 * row
-    b_d = 16 * 1024 * row * 2
-    out["ragged_16_B1024"] = {"tokens": sum(lens5), "compress_us": round(ms_c * 1e3, 2), "compress_kernels": nl_c,
-                              "ktok_s": round(sum(lens5) / (ms_c * 1e-3) / 1e3, 1), "compress_bytes": b_c,
-                              "compress": rate(b_c, ms_c, hbm), "decode_us": round(ms_d * 1e3, 2),
-                              "decode_bytes": b_d, "decode": rate(b_d, ms_d, hbm)}
-    del c5, d5, q5, k5, v5
+    if only in (None, "ragged"):
+        # -- ragged batch: 16 lengths uniform on [4096, 65536], B = min(1024, len), then decode over the 16 caches
+        lens5 = [int(x) for x in synth.ragged_lengths(1005, 16, 4096, 65536)]
+        q5, k5, v5 = device_inputs(seed + 5, lens5, n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
+        c5 = Compressor("bf16", lens5, n_h, n_kv, d, w, pk, 1024, device=dev, keep_raw=False)
+        cb5 = c5.buf.cu_budget_host
+        off5 = torch.tensor(cb5[:-1], dtype=torch.int64, device=dev)
+        ln5 = torch.tensor(np.diff(cb5), dtype=torch.int32, device=dev)
+        qd5 = torch.randn((16, n_h, d), device=dev).to(torch.bfloat16)
+        d5 = Decoder(16, n_h, n_kv, d, 1024, device=dev)
+        ms_c, mn_c, nl_c = time_graph([lambda: c5.compress(q5, k5, v5)], flush_l2, stream, steps)
+        ms_d, mn_d, nl_d = time_graph([lambda: d5.run(qd5, c5.buf.k_c, c5.buf.v_c, off5, ln5)], flush_l2, stream, steps)
+        b_c = sum(lens5) * row + 2 * 2 * 16 * 1024 * row
+        b_d = 16 * 1024 * row * 2
+        out["ragged_16_B1024"] = {"tokens": sum(lens5), "compress_us": round(ms_c * 1e3, 2), "compress_kernels": nl_c,
+                                  "ktok_s": round(sum(lens5) / (ms_c * 1e-3) / 1e3, 1), "compress_bytes": b_c,
+                                  "compress": rate(b_c, ms_c, hbm), "decode_us": round(ms_d * 1e3, 2),
+                                  "decode_bytes": b_d, "decode": rate(b_d, ms_d, hbm)}
+        del c5, d5, q5, k5, v5
 
-    # -- FreeKV decode step: batch 16 over full caches of S = 32768, B = 2048, tau = 0.9
-    S6, B6, nb6 = 32768, 2048, 16
-    _, k6, v6 = device_inputs(seed + 6, [S6] * nb6, n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
-    fk = FreeKvStep([S6] * nb6, n_h, n_kv, d, w, pk, B6, 0.9, device=dev)
-    q_prev = synth.decode_queries(seed + 61, nb6, n_h, d, "bf16")
-    q_cur = synth.drifted_queries(seed + 62, q_prev, "bf16", group=n_h // n_kv)
-    qp, qc = to_device(q_prev, "bf16", dev), to_device(q_cur, "bf16", dev)
-    fk.step(qp, qp, k6, v6, tau=2.0)                     # first step: every head selects
-    torch.cuda.synchronize()
-    idx0, kc0, vc0 = fk.idx.clone(), fk.k_c.clone(), fk.v_c.clone()
+    if only in (None, "freekv"):
+        # -- FreeKV decode step: batch 16 over full caches of S = 32768, B = 2048, tau = 0.9
+        S6, B6, nb6 = 32768, 2048, 16
+        _, k6, v6 = device_inputs(seed + 6, [S6] * nb6, n_h, n_kv, d, w, "bf16", 0.01, 3.0, dev)
+        fk = FreeKvStep([S6] * nb6, n_h, n_kv, d, w, pk, B6, 0.9, device=dev)
+        q_prev = synth.decode_queries(seed + 61, nb6, n_h, d, "bf16")
+        q_cur = synth.drifted_queries(seed + 62, q_prev, "bf16", group=n_h // n_kv)
+        qp, qc = to_device(q_prev, "bf16", dev), to_device(q_cur, "bf16", dev)
+        fk.step(qp, qp, k6, v6, tau=2.0)                     # first step: every head selects
+        torch.cuda.synchronize()
+        idx0, kc0, vc0 = fk.idx.clone(), fk.k_c.clone(), fk.v_c.clone()
 
-    def fk_step():
-        fk.idx.copy_(idx0)                               # every replay starts from the same previous step
-        fk.k_c.copy_(kc0)
-        fk.v_c.copy_(vc0)
-        fk.step(qc, qp, k6, v6)
-    ms, mn, nl = time_graph([fk_step], flush_l2, stream, steps)
-    # the restore copies are timed too; time them alone and subtract
-    ms_r, _, _ = time_graph([lambda: (fk.idx.copy_(idx0), fk.k_c.copy_(kc0), fk.v_c.copy_(vc0))], flush_l2, stream,
-                            steps)
-    n_flag = int(fk.reselected.sum().item())
-    b = n_flag * (S6 * 256 + 2 * 2 * B6 * 256) + nb6 * B6 * row * 2
-    ms_step = max(ms - ms_r, 1e-6)
-    out["freekv_step_b16_S32768_B2048"] = {"us": round(ms_step * 1e3, 2), "kernels": nl,
-                                           "reselected_heads": n_flag, "heads": nb6 * n_kv, "tau": 0.9,
-                                           "bytes": b, **rate(b, ms_step, hbm),
-                                           "note": "restore copies timed separately and subtracted"}
-    del fk, k6, v6
+        def fk_step():
+            fk.idx.copy_(idx0)                               # every replay starts from the same previous step
+            fk.k_c.copy_(kc0)
+            fk.v_c.copy_(vc0)
+            fk.step(qc, qp, k6, v6)
+        ms, mn, nl = time_graph([fk_step], flush_l2, stream, steps)
+        # the restore copies are timed too; time them alone and subtract
+        ms_r, _, _ = time_graph([lambda: (fk.idx.copy_(idx0), fk.k_c.copy_(kc0), fk.v_c.copy_(vc0))], flush_l2, stream,
+                                steps)
+        n_flag = int(fk.reselected.sum().item())
+        b = n_flag * (S6 * 256 + 2 * 2 * B6 * 256) + nb6 * B6 * row * 2
+        ms_step = max(ms - ms_r, 1e-6)
+        out["freekv_step_b16_S32768_B2048"] = {"us": round(ms_step * 1e3, 2), "kernels": nl,
+                                               "reselected_heads": n_flag, "heads": nb6 * n_kv, "tau": 0.9,
+                                               "bytes": b, **rate(b, ms_step, hbm),
+                                               "note": "restore copies timed separately and subtracted"}
+        del fk, k6, v6
 
-    # -- int8 compact caches: gather-and-quantise (16 x 2048 rows) and decode over them at batch 16
-    nb7, B7 = 16, 2048
-    kb = torch.randn((nb7 * B7, n_kv, d), device=dev).to(torch.bfloat16)
-    vb = torch.randn_like(kb)
-    idx7 = torch.arange(nb7 * B7, dtype=torch.int32, device=dev).repeat(n_kv, 1).contiguous()
-    cu7 = torch.tensor([0, nb7 * B7], dtype=torch.int32, device=dev)
-    kq = torch.empty((nb7 * B7, n_kv, d), dtype=torch.int8, device=dev)
-    vq = torch.empty_like(kq)
-    ks = torch.empty((n_kv, nb7 * B7), dtype=torch.float32, device=dev)
-    vs = torch.empty_like(ks)
-    ms_g, _, nl_g = time_graph([lambda: kvc.kvc_gather_kv_q8([nb7 * B7], cu7, cu7, nb7 * B7, idx7, kb, vb, kq, vq,
-                                                             ks, vs)], flush_l2, stream, steps)
-    qd7 = torch.randn((nb7, n_h, d), device=dev).to(torch.bfloat16)
-    off7 = torch.arange(nb7, dtype=torch.int64, device=dev) * B7
-    ln7 = torch.full((nb7,), B7, dtype=torch.int32, device=dev)
-    d7 = Decoder(nb7, n_h, n_kv, d, B7, device=dev)
-    ms_d, mn_d, nl_d = time_graph([lambda: kvc.kvc_gqa_decode_attn_q8(qd7, kq, vq, ks, vs, off7, ln7, B7, 0.0, d7.out,
-                                                                      d7.ws)], flush_l2, stream, steps)
-    rows = nb7 * B7 * n_kv
-    b_g = rows * (2 * 256 + 2 * 128 + 8)
-    b_d = rows * (2 * 128 + 8)
-    out["q8_b16_B2048"] = {"gather_quantise_us": round(ms_g * 1e3, 2), "gather_quantise_bytes": b_g,
-                           "gather_quantise": rate(b_g, ms_g, hbm), "decode_us": round(ms_d * 1e3, 2),
-                           "decode_bytes": b_d, "decode": rate(b_d, ms_d, hbm)}
-    del kb, vb, kq, vq, d7
+    if only in (None, "q8"):
+        # -- int8 compact caches: gather-and-quantise (16 x 2048 rows) and decode over them at batch 16
+        nb7, B7 = 16, 2048
+        kb = torch.randn((nb7 * B7, n_kv, d), device=dev).to(torch.bfloat16)
+        vb = torch.randn_like(kb)
+        idx7 = torch.arange(nb7 * B7, dtype=torch.int32, device=dev).repeat(n_kv, 1).contiguous()
+        cu7 = torch.tensor([0, nb7 * B7], dtype=torch.int32, device=dev)
+        kq = torch.empty((nb7 * B7, n_kv, d), dtype=torch.int8, device=dev)
+        vq = torch.empty_like(kq)
+        ks = torch.empty((n_kv, nb7 * B7), dtype=torch.float32, device=dev)
+        vs = torch.empty_like(ks)
+        ms_g, _, nl_g = time_graph([lambda: kvc.kvc_gather_kv_q8([nb7 * B7], cu7, cu7, nb7 * B7, idx7, kb, vb, kq, vq,
+                                                                 ks, vs)], flush_l2, stream, steps)
+        qd7 = torch.randn((nb7, n_h, d), device=dev).to(torch.bfloat16)
+        off7 = torch.arange(nb7, dtype=torch.int64, device=dev) * B7
+        ln7 = torch.full((nb7,), B7, dtype=torch.int32, device=dev)
+        d7 = Decoder(nb7, n_h, n_kv, d, B7, device=dev)
+        ms_d, mn_d, nl_d = time_graph([lambda: kvc.kvc_gqa_decode_attn_q8(qd7, kq, vq, ks, vs, off7, ln7, B7, 0.0, d7.out,
+                                                                          d7.ws)], flush_l2, stream, steps)
+        rows = nb7 * B7 * n_kv
+        b_g = rows * (2 * 256 + 2 * 128 + 8)
+        b_d = rows * (2 * 128 + 8)
+        out["q8_b16_B2048"] = {"gather_quantise_us": round(ms_g * 1e3, 2), "gather_quantise_bytes": b_g,
+                               "gather_quantise": rate(b_g, ms_g, hbm), "decode_us": round(ms_d * 1e3, 2),
+                               "decode_bytes": b_d, "decode": rate(b_d, ms_d, hbm)}
+        del kb, vb, kq, vq, d7
 
-    # -- xKV: factorise the keys of a window of W = 4 layers (S = 32768, r = 64, bf16 basis, 8 iteration steps),
-    #    then rebuild 2048 selected rows per head of one layer (selective) and all S rows (dense)
-    S8, W8, r8, it8 = 32768, 4, 64, 8
-    F8 = W8 * d
-    keys8 = [torch.randn((S8, n_kv, d), device=dev).to(torch.bfloat16) for _ in range(W8)]
-    gen8 = torch.Generator(device=dev)
-    gen8.manual_seed(seed + 8)
-    v08 = torch.randn((n_kv, F8, r8), generator=gen8, device=dev)
-    basis8 = torch.empty((n_kv, S8, r8), dtype=torch.bfloat16, device=dev)
-    blocks8 = torch.empty((n_kv, r8, F8), dtype=torch.float32, device=dev)
-    ws8 = torch.empty(kvc.kvc_xkv_workspace_size(S8, n_kv, d, W8, r8), dtype=torch.uint8, device=dev)
-    ms_f, _, nl_f = time_graph([lambda: kvc.kvc_xkv_factorize(keys8, r8, it8, v08, basis8, blocks8, ws8)], flush_l2,
-                               stream, steps)
-    gram_flops = 2 * S8 * F8 * F8 * n_kv
-    b_f = 2 * W8 * S8 * n_kv * d * 2 + n_kv * S8 * r8 * 2         # keys read by the Gram and the projection, A written
-    res = {"factorize_us": round(ms_f * 1e3, 2), "factorize_kernels": nl_f, "iters": it8,
-           "gram_tflops_equiv": round(gram_flops / (ms_f * 1e-3) / 1e12, 1), "factorize_bytes": b_f,
-           "factorize": rate(b_f, ms_f, hbm)}
-    for n_sel, tag in ((2048, "selective_2048"), (S8, "dense")):
-        idx8 = torch.randint(0, S8, (n_kv, n_sel), dtype=torch.int32, device=dev)
-        out8 = torch.empty((n_sel, n_kv, d), dtype=torch.bfloat16, device=dev)
-        ms_r, _, nl_r = time_graph([lambda: kvc.kvc_xkv_reconstruct(W8, 1, basis8, blocks8, idx8, out8)], flush_l2,
+    if only in (None, "xkv"):
+        # -- xKV: factorise the keys of a window of W = 4 layers (S = 32768, r = 64, bf16 basis, 8 iteration steps),
+        #    then rebuild 2048 selected rows per head of one layer (selective) and all S rows (dense)
+        S8, W8, r8, it8 = 32768, 4, 64, 8
+        F8 = W8 * d
+        keys8 = [torch.randn((S8, n_kv, d), device=dev).to(torch.bfloat16) for _ in range(W8)]
+        gen8 = torch.Generator(device=dev)
+        gen8.manual_seed(seed + 8)
+        v08 = torch.randn((n_kv, F8, r8), generator=gen8, device=dev)
+        basis8 = torch.empty((n_kv, S8, r8), dtype=torch.bfloat16, device=dev)
+        blocks8 = torch.empty((n_kv, r8, F8), dtype=torch.float32, device=dev)
+        ws8 = torch.empty(kvc.kvc_xkv_workspace_size(S8, n_kv, d, W8, r8), dtype=torch.uint8, device=dev)
+        ms_f, _, nl_f = time_graph([lambda: kvc.kvc_xkv_factorize(keys8, r8, it8, v08, basis8, blocks8, ws8)], flush_l2,
                                    stream, steps)
-        b_r = n_sel * n_kv * (r8 * 2 + d * 2 + 4) + n_kv * r8 * d * 4
-        res[f"rebuild_{tag}_us"] = round(ms_r * 1e3, 2)
-        res[f"rebuild_{tag}_bytes"] = b_r
-        res[f"rebuild_{tag}"] = rate(b_r, ms_r, hbm)
-        res[f"rebuild_{tag}_gflops"] = round(2 * n_sel * n_kv * r8 * d / (ms_r * 1e-3) / 1e9, 1)
-        del idx8, out8
-    out[f"xkv_S{S8}_W{W8}_r{r8}"] = res
-    del keys8, v08, basis8, blocks8, ws8
+        gram_flops = 2 * S8 * F8 * F8 * n_kv
+        b_f = 2 * W8 * S8 * n_kv * d * 2 + n_kv * S8 * r8 * 2         # keys read by the Gram and the projection, A written
+        res = {"factorize_us": round(ms_f * 1e3, 2), "factorize_kernels": nl_f, "iters": it8,
+               "gram_tflops_equiv": round(gram_flops / (ms_f * 1e-3) / 1e12, 1), "factorize_bytes": b_f,
+               "factorize": rate(b_f, ms_f, hbm)}
+        for n_sel, tag in ((2048, "selective_2048"), (S8, "dense")):
+            idx8 = torch.randint(0, S8, (n_kv, n_sel), dtype=torch.int32, device=dev)
+            out8 = torch.empty((n_sel, n_kv, d), dtype=torch.bfloat16, device=dev)
+            ms_r, _, nl_r = time_graph([lambda: kvc.kvc_xkv_reconstruct(W8, 1, basis8, blocks8, idx8, out8)], flush_l2,
+                                       stream, steps)
+            b_r = n_sel * n_kv * (r8 * 2 + d * 2 + 4) + n_kv * r8 * d * 4
+            res[f"rebuild_{tag}_us"] = round(ms_r * 1e3, 2)
+            res[f"rebuild_{tag}_bytes"] = b_r
+            res[f"rebuild_{tag}"] = rate(b_r, ms_r, hbm)
+            res[f"rebuild_{tag}_gflops"] = round(2 * n_sel * n_kv * r8 * d / (ms_r * 1e-3) / 1e9, 1)
+            del idx8, out8
+        out[f"xkv_S{S8}_W{W8}_r{r8}"] = res
+        del keys8, v08, basis8, blocks8, ws8
+
     torch.cuda.empty_cache()
     return out
 
@@ -752,6 +763,28 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_one_workload(args):
+    """One workload of the set on one GPU, alone, printed as one JSON line."""
+    import torch
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    from kv_cache_compression_score_b200 import build as kbuild
+    kbuild.build()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sweep = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        torch.sum(sweep, dim=0, out=sink)
+
+    hbm, peak_kind = measured_peaks()
+    res = run_workloads(args, dev, torch.cuda.current_stream(dev), flush_l2, LLAMA3_8B_S32K["seed"], hbm,
+                        only=args.workload)
+    print(json.dumps({"workload": args.workload, "peak_gbs": hbm, "peak_kind": peak_kind, "steps": args.steps,
+                      "warmup": args.warmup, "results": res}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -760,11 +793,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--headline-only", action="store_true",
                     help="time only the Llama-3-8B S=32K layer (skip the other workloads)")
+    ap.add_argument("--workload", choices=WORKLOAD_NAMES, default=None,
+                    help="time only this one workload of the set (no headline line; for profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload:
+        run_one_workload(args)
     else:
         run_ours(args)
 
