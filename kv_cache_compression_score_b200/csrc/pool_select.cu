@@ -297,11 +297,11 @@ KVC_DEVINL void cluster_topk_adaptive(const float *__restrict__ src, int n, int 
 
 // Block-wide radix select over keys[0..n) in shared memory (one CTA): the
 // k-th largest key T and how many keys equal to T are among the k largest.
-KVC_DEVINL void block_kth_largest(const uint32_t *keys, int n, int k, CSel &sm, uint32_t *T_out, int *take_eq) {
+KVC_DEVINL void block_kth_largest(const uint32_t *keys, int n, int k, CSel &sm, uint32_t *T_out, int *take_eq,
+                                  int hi_bit = 31, uint32_t prefix = 0u, uint32_t pmask = 0u) {
   const int tid = threadIdx.x;
-  uint32_t prefix = 0u, pmask = 0u;
   int k_rem = k;
-  for (int hi = 31; hi >= 0; hi -= 11) {
+  for (int hi = hi_bit; hi >= 0; hi -= 11) {
     const int width = min(11, hi + 1), shift = hi + 1 - width, nb = 1 << width;
     int *H = sm.hist[1];
     for (int i = tid; i < nb; i += kCThreads) H[i] = 0;
@@ -338,9 +338,9 @@ KVC_DEVINL void block_kth_largest(const uint32_t *keys, int n, int k, CSel &sm, 
 // [2^-30, 2^34), lower scores (and negative ones) in bin 0, higher in bin 2047.
 // Monotone in the key, so whole buckets above the threshold bucket are
 // selected and whole buckets below are not.
+KVC_DEVINL constexpr int top_digit_lo() { return (int)((0x80000000u | (97u << 23)) >> 18); }   // key of 2^-30 / 2^18
 KVC_DEVINL int top_digit(uint32_t u) {
-  constexpr int kLo = (int)((0x80000000u | (97u << 23)) >> 18);   // key of 2^-30, in units of 2^18
-  const int d = (int)(u >> 18) - kLo;
+  const int d = (int)(u >> 18) - top_digit_lo();
   return d < 0 ? 0 : (d > kCBins - 1 ? kCBins - 1 : d);
 }
 
@@ -407,11 +407,21 @@ KVC_DEVINL void cluster_topk_ascending(const float *__restrict__ src, int n, int
   __syncthreads();
   const int bstar = sm.sel[0], above = sm.sel[1];      // keys in bins > bstar (whole cluster)
   // this CTA's candidates: its keys in bucket bstar
-  for (int i = beg; i < end; ++i) {
-    const uint32_t u = cache[i + (i >> 5)];
-    if (top_digit(u) == bstar) {
-      const int slot = atomicAdd(&sm.ncand, 1);
-      if (slot < kCandLocal) sm.cand[slot] = u;
+  // (one shared atomic per warp and step: the lanes holding a candidate take
+  // consecutive slots)
+  for (int q = 0; q < E; ++q) {
+    const int i = beg + q;
+    const uint32_t u = i < end ? cache[i + (i >> 5)] : 0u;
+    const bool c = i < end && top_digit(u) == bstar;
+    const uint32_t m = __ballot_sync(0xffffffffu, c);
+    if (m) {
+      int base = 0;
+      if (lane_id() == __ffs(m) - 1) base = atomicAdd(&sm.ncand, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+      if (c) {
+        const int slot = base + __popc(m & ((1u << lane_id()) - 1u));
+        if (slot < kCandLocal) sm.cand[slot] = u;
+      }
     }
   }
   cluster_sync_all();                                   // (2) every CTA's candidates are listed
@@ -475,6 +485,10 @@ KVC_DEVINL void cluster_topk_ascending(const float *__restrict__ src, int n, int
     __syncthreads();
     T = (uint32_t)sm.sel[2];
     take_eq = sm.sel[3];
+  } else if (bstar > 0 && bstar < kCBins - 1) {
+    // every candidate has the 14 key bits 31..18 of bucket bstar
+    const uint32_t hi14 = ((uint32_t)(bstar + top_digit_lo()) << 18);
+    block_kth_largest(sm.all, total, k_rem, sm, &T, &take_eq, 17, hi14, 0xfffc0000u);
   } else {
     block_kth_largest(sm.all, total, k_rem, sm, &T, &take_eq);
   }

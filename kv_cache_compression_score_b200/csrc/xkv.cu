@@ -27,9 +27,10 @@
 //               leaves C zero for the next step;
 //   xkv_apply   32 rows of V = Y M per CTA (float64 products); the last step
 //               also writes Vt;
-//   xkv_project A_h = X_h V, 64 tokens per CTA, V in shared memory;
-//   xkv_rebuild rows idx of layer l: A_h[idx] Vt_h[:, layer block], rounded to
-//               bf16 (nearest even).
+//   xkv_project_tc A_h = X_h V on the tensor cores (V split into two bf16
+//               terms), a run of 128-token tiles per CTA;
+//   xkv_rebuild_tc rows idx of layer l: A_h[idx] Vt_h[:, layer block] on the
+//               tensor cores, rounded to bf16 (nearest even).
 #include <algorithm>
 
 #include "kvc_common.cuh"
@@ -39,7 +40,8 @@ namespace kvc {
 namespace {
 
 constexpr int kGramTile = 64;     // output tile of the Gram kernel
-constexpr int kGramS = 32;        // tokens per pipeline step
+constexpr int kGramS = 64;        // tokens per pipeline stage
+constexpr int kGramStages = 4;    // cp.async ring depth of the Gram kernel
 constexpr int kGramPitch = 72;    // bf16 per padded smem row (144 bytes: the 8 rows of an ldmatrix hit distinct banks)
 constexpr int kRowsPerCta = 32;   // xkv_gv / xkv_apply
 constexpr int kGvK = 64;          // xkv_gv: rows k of G and V per pipeline step
@@ -55,7 +57,6 @@ struct XkArgs {
   double *m;                      // [n_kv, r, r] upper triangular L^-T
   float *v_out;                   // [n_kv, F, r]
   float *blocks;                  // Vt [n_kv, r, F] (written by the last apply)
-  const float *v_final;           // [n_kv, F, r] for the projection
   void *basis;                    // A [n_kv, S, r], float32 or bf16
   bool basis_bf16;
 };
@@ -67,9 +68,12 @@ KVC_DEVINL const __nv_bfloat16 *xptr(const XkArgs &a, int h, int s, int f) {
 }
 
 // ------------------------------------------------------------------ Gram
+constexpr int kGramSmem = 2 * kGramStages * kGramS * kGramPitch * 2;
+
 __global__ void __launch_bounds__(128) xkv_gram(XkArgs a) {
-  __shared__ __align__(16) __nv_bfloat16 si[2][kGramS][kGramPitch];
-  __shared__ __align__(16) __nv_bfloat16 sj[2][kGramS][kGramPitch];
+  extern __shared__ __align__(16) uint8_t xk_gram_smem[];
+  auto si = reinterpret_cast<__nv_bfloat16 (*)[kGramS][kGramPitch]>(xk_gram_smem);
+  auto sj = reinterpret_cast<__nv_bfloat16 (*)[kGramS][kGramPitch]>(xk_gram_smem + kGramSmem / 2);
   // upper-triangular tile pair (ti <= tj) from blockIdx.x
   const int nt = a.F / kGramTile;
   int ti = 0, rem = blockIdx.x;
@@ -100,16 +104,20 @@ __global__ void __launch_bounds__(128) xkv_gram(XkArgs a) {
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  // ring of kGramStages stages: stage st is in buffer st % kGramStages; one
+  // commit group per stage (empty past the end), so that waiting until at
+  // most kGramStages - 1 groups are pending means stage st has landed
   const int n_steps = (s1 - s0 + kGramS - 1) / kGramS;
-  load(0, s0);
+  for (int q = 0; q < kGramStages - 1; ++q) {
+    if (q < n_steps) load(q, s0 + q * kGramS);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+  }
   for (int st = 0; st < n_steps; ++st) {
-    const int buf = st & 1;
-    if (st + 1 < n_steps) {
-      load(buf ^ 1, s0 + (st + 1) * kGramS);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
+    const int buf = st % kGramStages;
+    const int nx = st + kGramStages - 1;
+    if (nx < n_steps) load(nx % kGramStages, s0 + nx * kGramS);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group %0;" :: "n"(kGramStages - 1) : "memory");
     __syncthreads();
 #pragma unroll
     for (int ks = 0; ks < kGramS / 16; ++ks) {
@@ -194,8 +202,16 @@ __global__ void __launch_bounds__(128) xkv_gv(XkArgs a) {
     for (int kk = 0; kk < kGvK; ++kk) {
       const float4 g4 = *reinterpret_cast<const float4 *>(g_t + kk * kRowsPerCta);
       float vv[CPT];
+      if constexpr (CPT == 4) {
+        const float4 v4 = *reinterpret_cast<const float4 *>(v_t + kk * R);
+        vv[0] = v4.x; vv[1] = v4.y; vv[2] = v4.z; vv[3] = v4.w;
+      } else if constexpr (CPT == 2) {
+        const float2 v2 = *reinterpret_cast<const float2 *>(v_t + kk * R);
+        vv[0] = v2.x; vv[1] = v2.y;
+      } else {
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) vv[c] = v_t[kk * R + c];
+        for (int c = 0; c < CPT; ++c) vv[c] = v_t[kk * R + c];
+      }
 #pragma unroll
       for (int c = 0; c < CPT; ++c) {
         acc[0][c] = fmaf(g4.x, vv[c], acc[0][c]);
@@ -230,54 +246,116 @@ __global__ void __launch_bounds__(128) xkv_gv(XkArgs a) {
 }
 
 // ------------------------------------------------ Cholesky and M = L^-T
-// One CTA per head, 256 threads.  Right-looking Cholesky of C with two
-// barriers per column, then L^-1 row by row (4 threads per column, their
-// partial sums combined by shuffles), stored transposed as M.
+// 1 / sqrt(x) in float64: the float32 reciprocal square root as a seed (about
+// 22 correct bits), then two Newton-Raphson steps y <- y (3 - x y^2) / 2, each
+// doubling the correct bits (22 -> 44 -> past the 53 of a double).  Values
+// outside the float32 range take the plain quotient.
+KVC_DEVINL double rsqrt_newton(double x) {
+  if (!(x > 1e-37 && x < 1e37)) return 1.0 / sqrt(x);
+  double y = (double)rsqrtf((float)x);
+  y = y * fma(-0.5 * x * y, y, 1.5);
+  y = y * fma(-0.5 * x * y, y, 1.5);
+  return y;
+}
+
+// One CTA per head, 512 threads, one barrier per column and one per four
+// rows of the inverse.  Column c of L is written from the unscaled working
+// copy in the same phase as the rank-1 update of the trailing block (thread
+// (tp, tq) updates rows tp, tp + 16, .. and columns tq, tq + 32, ..), so no
+// phase reads what it writes.  L^-1 is formed four rows at a time: 8 threads
+// per column sum the terms of the rows above the block, and one of them
+// finishes the 4 x 4 triangular block; it is stored transposed as M.  Pivots
+// are inverted once (by the thread that finished them) and multiplied.
 template <int R>
-__global__ void __launch_bounds__(256) xkv_chol(XkArgs a) {
+__global__ void __launch_bounds__(512) xkv_chol(XkArgs a) {
   constexpr int LP = R + 1;
   extern __shared__ __align__(16) double xk_chol_smem[];
-  double *L = xk_chol_smem;          // [R][LP]
-  double *X = L + R * LP;            // [R][LP]: L^-1
-  double *diag = X + R * LP;         // [R]
+  double *A = xk_chol_smem;          // [R][LP] working copy, updated in place
+  double *L = A + R * LP;            // [R][LP] strictly lower part of the factor
+  double *X = L + R * LP;            // [R][LP] L^-1
+  double *dinv = X + R * LP;         // [R]: 1 / L[c][c]
   const int h = blockIdx.x, tid = threadIdx.x;
   double *C = a.c + (size_t)h * R * R;
-  for (int e = tid; e < R * R; e += 256) {
+  for (int e = tid; e < R * R; e += 512) {
     const int p = e / R, q = e % R;
-    L[p * LP + q] = q <= p ? C[e] : 0.0;
+    A[p * LP + q] = q <= p ? C[e] : 0.0;
     X[p * LP + q] = 0.0;
     C[e] = 0.0;                      // ready for the next step's atomics
   }
   __syncthreads();
   double tr = 0.0;
-  for (int p = 0; p < R; ++p) tr += L[p * LP + p];
+  for (int p = 0; p < R; ++p) tr += A[p * LP + p];
   // a pivot below this floor (a rank-deficient Y) is raised to it
   const double floor_piv = fmax(tr, 1e-300) * 1e-30;
+  if (tid == 0) dinv[0] = rsqrt_newton(fmax(A[0], floor_piv));
+  __syncthreads();
+  const int tp = tid >> 5, tq = tid & 31;
+  constexpr int NP = (R + 15) / 16, NQ = (R + 31) / 32;
   for (int c = 0; c < R; ++c) {
-    const double dcc = sqrt(fmax(L[c * LP + c], floor_piv));
-    if (tid == 0) diag[c] = dcc;
-    for (int p = c + 1 + tid; p < R; p += 256) L[p * LP + c] /= dcc;
+    const double inv = dinv[c];
+    if (c + 1 + tid < R) L[(c + 1 + tid) * LP + c] = A[(c + 1 + tid) * LP + c] * inv;
+    // the column-c values this thread needs, loaded before any update
+    double lq[NQ], lp[NP];
+#pragma unroll
+    for (int qi = 0; qi < NQ; ++qi) {
+      const int q = c + 1 + tq + 32 * qi;
+      lq[qi] = q < R ? A[q * LP + c] : 0.0;
+    }
+#pragma unroll
+    for (int pi = 0; pi < NP; ++pi) {
+      const int p = c + 1 + tp + 16 * pi;
+      lp[pi] = p < R ? A[p * LP + c] * inv * inv : 0.0;
+    }
+#pragma unroll
+    for (int pi = 0; pi < NP; ++pi) {
+      const int p = c + 1 + tp + 16 * pi;
+#pragma unroll
+      for (int qi = 0; qi < NQ; ++qi) {
+        const int q = c + 1 + tq + 32 * qi;
+        if (p < R && q <= p) A[p * LP + q] = fma(-lp[pi], lq[qi], A[p * LP + q]);
+      }
+    }
+    // thread 0 owns (c + 1, c + 1): no other thread writes it in this phase
+    if (tid == 0 && c + 1 < R) dinv[c + 1] = rsqrt_newton(fmax(A[(c + 1) * LP + c + 1], floor_piv));
     __syncthreads();
-    const int n = R - c - 1;
-    for (int e = tid; e < n * n; e += 256) {
-      const int p = c + 1 + e / n, q = c + 1 + e % n;
-      if (q <= p) L[p * LP + q] -= L[p * LP + c] * L[q * LP + c];
+  }
+  // X = L^-1 (lower), rows i0 .. i0 + 3 per step; thread group (j, part)
+  const int j = tid >> 3, part = tid & 7;
+  for (int i0 = 0; i0 < R; i0 += 4) {
+    double s[4] = {0.0, 0.0, 0.0, 0.0};
+    if (j < i0)
+      for (int k = j + part; k < i0; k += 8) {
+        const double xk = X[k * LP + j];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) s[r] = fma(L[(i0 + r) * LP + k], xk, s[r]);
+      }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      s[r] += __shfl_xor_sync(0xffffffffu, s[r], 1);
+      s[r] += __shfl_xor_sync(0xffffffffu, s[r], 2);
+      s[r] += __shfl_xor_sync(0xffffffffu, s[r], 4);
+    }
+    if (part == 0 && j < i0 + 4) {
+      double xb[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = i0 + r;
+        double v = 0.0;
+        if (j == i) {
+          v = dinv[i];
+        } else if (j < i) {
+          double sum = s[r];
+          for (int k = max(j, i0); k < i; ++k) sum = fma(L[i * LP + k], xb[k - i0], sum);
+          v = -sum * dinv[i];
+        }
+        xb[r] = v;
+        X[i * LP + j] = v;
+      }
     }
     __syncthreads();
   }
-  // X = L^-1 (lower), row i from rows < i; thread group (j, part), j < R
-  const int j = tid / 4, part = tid % 4;
-  for (int i = 0; i < R; ++i) {
-    double s = 0.0;
-    if (j < i)
-      for (int k = j + part; k < i; k += 4) s = fma(L[i * LP + k], X[k * LP + j], s);
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    if (part == 0 && j <= i) X[i * LP + j] = j == i ? 1.0 / diag[i] : -s / diag[i];
-    __syncthreads();
-  }
   double *M = a.m + (size_t)h * R * R;
-  for (int e = tid; e < R * R; e += 256) {
+  for (int e = tid; e < R * R; e += 512) {
     const int k = e / R, c = e % R;
     M[e] = X[c * LP + k];            // M[k][c] = (L^-1)[c][k], zero for k > c
   }
@@ -307,72 +385,115 @@ __global__ void __launch_bounds__(128) xkv_apply(XkArgs a, int write_blocks) {
 }
 
 // ------------------------------------------------------------ A = X V
+// Tensor cores: A (tokens x r) = X (tokens x F, bf16, exact) times V (F x r)
+// with V = Vt^T split into two bf16 terms (v = hi + lo, |v - hi - lo| <=
+// 2^-17 |v|), mma.sync m16n8k16 with fp32 accumulation.  A CTA stages both
+// terms of Vt ([r][F], F contiguous) once and walks a contiguous run of
+// 128-token tiles; each tile's X streams in 64-feature chunks through two
+// cp.async buffers.  Warp w owns tokens 16w .. 16w + 15 of a tile and all r
+// columns.
+constexpr int kPjTok = 128;       // tokens per tile
+constexpr int kPjK = 64;          // features per chunk
+constexpr int kPjXP = kPjK + 8;   // bf16 pitch of an X chunk row (144 B)
+
 template <int R>
-__global__ void __launch_bounds__(256) xkv_project(XkArgs a) {
-  extern __shared__ __align__(16) float xk_proj_smem[];
-  constexpr int CPT = R / 16;
-  float *sv = xk_proj_smem;                       // [F][R]
-  float *sx = xk_proj_smem + (size_t)a.F * R;     // [64][33]: 32 features of 64 tokens
-  const int h = blockIdx.y, s0 = blockIdx.x * 64, F = a.F;
-  const float *V = a.v_final + (size_t)h * F * R;
-  for (int e = threadIdx.x; e < F * R / 4; e += blockDim.x)
-    reinterpret_cast<float4 *>(sv)[e] = reinterpret_cast<const float4 *>(V)[e];
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;   // rows 4 ty .. 4 ty + 3, columns tx * CPT ..
-  float acc[4][CPT];
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[q][c] = 0.f;
-  for (int f0 = 0; f0 < F; f0 += 32) {
-    __syncthreads();
-    {   // 64 tokens x 4 pieces of 8 features: one piece per thread
-      const int row = threadIdx.x / 4, p8 = threadIdx.x % 4, s = s0 + row;
-      float vals[8];
-      if (s < a.S) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(xptr(a, h, s, f0 + 8 * p8));
-        Elem<__nv_bfloat16>::unpack(u, vals);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) vals[q] = 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sx[row * 33 + 8 * p8 + q] = vals[q];
+__global__ void __launch_bounds__(256) xkv_project_tc(XkArgs a, int tiles_per_cta) {
+  extern __shared__ __align__(16) uint8_t xk_proj_smem[];
+  const int F = a.F, VP = F + 8;                       // bf16 pitch of a Vt row
+  __nv_bfloat16 *vhi = reinterpret_cast<__nv_bfloat16 *>(xk_proj_smem);   // [R][VP]
+  __nv_bfloat16 *vlo = vhi + R * VP;
+  __nv_bfloat16 *xs = vlo + R * VP;                                       // [2][kPjTok][kPjXP]
+  const int h = blockIdx.y, warp = warp_id(), lane = lane_id();
+  const int n_tiles = (a.S + kPjTok - 1) / kPjTok;
+  const int tile0 = blockIdx.x * tiles_per_cta, tile1 = min(n_tiles, tile0 + tiles_per_cta);
+  if (tile0 >= tile1) return;
+  const int n_chunks = F / kPjK, n_items = (tile1 - tile0) * n_chunks;
+  auto load = [&](int item, int buf) {
+    const int tile = tile0 + item / n_chunks, f0 = (item % n_chunks) * kPjK;
+    for (int e = threadIdx.x; e < kPjTok * (kPjK / 8); e += 256) {
+      const int row = e / (kPjK / 8), c8 = e % (kPjK / 8), s = tile * kPjTok + row;
+      const bool ok = s < a.S;
+      cp_async16(xs + ((size_t)buf * kPjTok + row) * kPjXP + 8 * c8, xptr(a, h, ok ? s : 0, f0 + 8 * c8), ok);
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int ff = 0; ff < 32; ++ff) {
-      float xv[4];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  load(0, 0);
+  // both terms of Vt (overlaps the first chunk's copies)
+  const float *vt = a.blocks + (size_t)h * R * F;
+  for (int e = threadIdx.x; e < R * F / 4; e += 256) {
+    const int c = (4 * e) / F, f = (4 * e) % F;
+    const float4 v = *reinterpret_cast<const float4 *>(vt + (size_t)c * F + f);
+    const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) xv[q] = sx[(ty * 4 + q) * 33 + ff];
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        const float vv = sv[(f0 + ff) * R + tx * CPT + c];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[q][c] = fmaf(xv[q], vv, acc[q][c]);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(vv[q]);
+      vhi[c * VP + f + q] = hi;
+      vlo[c * VP + f + q] = __float2bfloat16_rn(vv[q] - __bfloat162float(hi));
     }
   }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int s = s0 + ty * 4 + q;
-    if (s >= a.S) continue;
-    const size_t o = ((size_t)h * a.S + s) * R + tx * CPT;
-    if (a.basis_bf16) {
-      __nv_bfloat16 *b = static_cast<__nv_bfloat16 *>(a.basis) + o;
-#pragma unroll
-      for (int c = 0; c < CPT; ++c) b[c] = __float2bfloat16_rn(acc[q][c]);
+  constexpr int NT = R / 8;                 // n8 tiles
+  const int g = lane >> 2, t = lane & 3, lr = lane & 7, li = lane >> 3;
+  float acc[NT][4];
+  for (int item = 0; item < n_items; ++item) {
+    const int buf = item & 1, chunk = item % n_chunks;
+    if (item + 1 < n_items) {
+      load(item + 1, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
-      float *b = static_cast<float *>(a.basis) + o;
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    if (chunk == 0) {
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) b[c] = acc[q][c];
+      for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    }
+    const __nv_bfloat16 *xb = xs + (size_t)buf * kPjTok * kPjXP;
+#pragma unroll
+    for (int ks = 0; ks < kPjK / 16; ++ks) {
+      uint32_t af[4];
+      ldsm_x4(smem_u32(xb + (16 * warp + lr + (li & 1) * 8) * kPjXP + 16 * ks + (li >> 1) * 8), af);
+      const int fk = chunk * kPjK + 16 * ks;
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        uint32_t bh[4], bl[4];
+        const int off = (16 * np + lr + (li >> 1) * 8) * VP + fk + (li & 1) * 8;
+        ldsm_x4(smem_u32(vhi + off), bh);
+        ldsm_x4(smem_u32(vlo + off), bl);
+        mma_bf16(acc[2 * np], af, bh[0], bh[1]);
+        mma_bf16(acc[2 * np], af, bl[0], bl[1]);
+        mma_bf16(acc[2 * np + 1], af, bh[2], bh[3]);
+        mma_bf16(acc[2 * np + 1], af, bl[2], bl[3]);
+      }
+    }
+    __syncthreads();
+    if (chunk == n_chunks - 1) {
+      const int tile = tile0 + item / n_chunks;
+#pragma unroll
+      for (int hi8 = 0; hi8 < 2; ++hi8) {
+        const int s = tile * kPjTok + 16 * warp + g + 8 * hi8;
+        if (s >= a.S) continue;
+        const size_t o = ((size_t)h * a.S + s) * R + 2 * t;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const float x0 = acc[n][2 * hi8], x1 = acc[n][2 * hi8 + 1];
+          if (a.basis_bf16)
+            *reinterpret_cast<uint32_t *>(static_cast<__nv_bfloat16 *>(a.basis) + o + 8 * n) = pack_bf16(x0, x1);
+          else
+            *reinterpret_cast<float2 *>(static_cast<float *>(a.basis) + o + 8 * n) = make_float2(x0, x1);
+        }
+      }
     }
   }
 }
 
 // ------------------------------------------------- selective reconstruction
-// CTA = (64 selected rows, head); the layer's r x d_h block of Vt in shared
-// memory; one warp per row, each lane d_h / 32 output dims; the basis row is
-// spread over the lanes and broadcast by shuffles.
+// CTA = (64 selected rows, head), 256 threads, on the tensor cores.  The
+// layer's r x d_h block of Vt is split into two bf16 terms in shared memory
+// ([c][j], j contiguous: the B operand through ldmatrix.trans); the 64 basis
+// rows are gathered with cp.async (bf16 basis, exact) or loaded and split into
+// two bf16 terms (float32 basis).  out = A . (Vt_hi + Vt_lo) [+ A_lo . Vt_hi]
+// with mma.sync m16n8k16 and fp32 accumulation, rounded to bf16.  Warp w owns
+// rows 16 (w & 3) .. + 15 and output dims (w >> 2) D/2 .. + D/2.
 struct XrArgs {
   int S, n_kv, d, F, layer, n_sel;
   const void *basis;
@@ -381,63 +502,109 @@ struct XrArgs {
   __nv_bfloat16 *out;
 };
 
+template <int R, int D>
+struct RebuildLayout {
+  static constexpr int BP = D + 8;            // bf16 pitch of a Vt block row
+  static constexpr int AP = R + 8;            // bf16 pitch of a basis row
+  static constexpr int kOffBl = R * BP * 2;
+  static constexpr int kOffAh = 2 * R * BP * 2;
+  static constexpr int kOffAl = kOffAh + 64 * AP * 2;
+  static constexpr int kOffIdx = kOffAl + 64 * AP * 2;
+  static constexpr int kBytes = kOffIdx + 64 * 4;
+};
+
 template <int R, int D, bool BF16>
-__global__ void __launch_bounds__(256) xkv_rebuild(XrArgs a) {
-  constexpr int DPL = D / 32;
-  constexpr int NU = (R + 31) / 32;
-  __shared__ __align__(16) float sb[R * D];
-  const int h = blockIdx.y, t0 = blockIdx.x * 64;
-  const float *vt = a.blocks + (size_t)h * R * a.F + (size_t)a.layer * D;
-  for (int e = threadIdx.x; e < R * D / 4; e += 256) {
-    const int c = e / (D / 4), j4 = e % (D / 4);
-    reinterpret_cast<float4 *>(sb)[e] = *reinterpret_cast<const float4 *>(vt + (size_t)c * a.F + 4 * j4);
+__global__ void __launch_bounds__(256) xkv_rebuild_tc(XrArgs a) {
+  using Ly = RebuildLayout<R, D>;
+  constexpr int BP = Ly::BP, AP = Ly::AP;
+  extern __shared__ __align__(16) uint8_t xk_rb_smem[];
+  __nv_bfloat16 *bh = reinterpret_cast<__nv_bfloat16 *>(xk_rb_smem);
+  __nv_bfloat16 *bl = reinterpret_cast<__nv_bfloat16 *>(xk_rb_smem + Ly::kOffBl);
+  __nv_bfloat16 *ah = reinterpret_cast<__nv_bfloat16 *>(xk_rb_smem + Ly::kOffAh);
+  __nv_bfloat16 *al = reinterpret_cast<__nv_bfloat16 *>(xk_rb_smem + Ly::kOffAl);
+  int *sidx = reinterpret_cast<int *>(xk_rb_smem + Ly::kOffIdx);
+  const int h = blockIdx.y, t0 = blockIdx.x * 64, tid = threadIdx.x;
+  if (tid < 64) {
+    const int t = t0 + tid;
+    const int src = t < a.n_sel ? __ldg(a.idx + (size_t)h * a.n_sel + t) : -1;
+    sidx[tid] = (src >= 0 && src < a.S) ? src : -1;
   }
   __syncthreads();
-  const int lane = lane_id();
-  const int t_end = min(a.n_sel, t0 + 64);
-  for (int t = t0 + warp_id(); t < t_end; t += 8) {
-    const int src = __ldg(a.idx + (size_t)h * a.n_sel + t);
-    const bool in = src >= 0 && src < a.S;
-    float av[NU];
-#pragma unroll
-    for (int u = 0; u < NU; ++u) {
-      const int c = lane + 32 * u;
-      float x = 0.f;
-      if (in && c < R) {
-        const size_t o = ((size_t)h * a.S + src) * R + c;
-        if constexpr (BF16) x = __bfloat162float(static_cast<const __nv_bfloat16 *>(a.basis)[o]);
-        else x = static_cast<const float *>(a.basis)[o];
-      }
-      av[u] = x;
+  // the 64 basis rows
+  if constexpr (BF16) {
+    const __nv_bfloat16 *base = static_cast<const __nv_bfloat16 *>(a.basis);
+    for (int e = tid; e < 64 * (R / 8); e += 256) {
+      const int row = e / (R / 8), p8 = e % (R / 8), src = sidx[row];
+      cp_async16(ah + row * AP + 8 * p8, base + ((size_t)h * a.S + (src < 0 ? 0 : src)) * R + 8 * p8, src >= 0);
     }
-    float acc[DPL];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  } else {
+    const float *base = static_cast<const float *>(a.basis);
+    for (int e = tid; e < 64 * (R / 4); e += 256) {
+      const int row = e / (R / 4), p4 = e % (R / 4), src = sidx[row];
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (src >= 0) v = __ldg(reinterpret_cast<const float4 *>(base + ((size_t)h * a.S + src) * R + 4 * p4));
+      const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int q = 0; q < DPL; ++q) acc[q] = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < R; ++c) {
-      const float ac = __shfl_sync(0xffffffffu, av[c / 32], c % 32);
-      const float *row = sb + c * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const float4 b4 = *reinterpret_cast<const float4 *>(row);
-        acc[0] = fmaf(ac, b4.x, acc[0]);
-        acc[1] = fmaf(ac, b4.y, acc[1]);
-        acc[2] = fmaf(ac, b4.z, acc[2]);
-        acc[3] = fmaf(ac, b4.w, acc[3]);
-      } else {
-        const float2 b2 = *reinterpret_cast<const float2 *>(row);
-        acc[0] = fmaf(ac, b2.x, acc[0]);
-        acc[1] = fmaf(ac, b2.y, acc[1]);
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(vv[q]);
+        ah[row * AP + 4 * p4 + q] = hi;
+        al[row * AP + 4 * p4 + q] = __float2bfloat16_rn(vv[q] - __bfloat162float(hi));
       }
     }
-    __nv_bfloat16 *o = a.out + ((size_t)t * a.n_kv + h) * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      uint2 u;
-      u.x = pack_bf16(acc[0], acc[1]);
-      u.y = pack_bf16(acc[2], acc[3]);
-      *reinterpret_cast<uint2 *>(o) = u;
-    } else {
-      *reinterpret_cast<uint32_t *>(o) = pack_bf16(acc[0], acc[1]);
+  }
+  // the layer's block of Vt, two terms
+  const float *vt = a.blocks + (size_t)h * R * a.F + (size_t)a.layer * D;
+  for (int e = tid; e < R * D / 4; e += 256) {
+    const int c = e / (D / 4), j4 = e % (D / 4);
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(vt + (size_t)c * a.F + 4 * j4));
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(vv[q]);
+      bh[c * BP + 4 * j4 + q] = hi;
+      bl[c * BP + 4 * j4 + q] = __float2bfloat16_rn(vv[q] - __bfloat162float(hi));
     }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  constexpr int NTW = D / 16;                 // n8 tiles per warp
+  const int warp = warp_id(), lane = lane_id();
+  const int mt = warp & 3, n0 = (warp >> 2) * (D / 2);
+  const int g = lane >> 2, t = lane & 3, lr = lane & 7, li = lane >> 3;
+  float acc[NTW][4];
+#pragma unroll
+  for (int n = 0; n < NTW; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < R / 16; ++ks) {
+    uint32_t af[4], afl[4];
+    const int aoff = (16 * mt + lr + (li & 1) * 8) * AP + 16 * ks + (li >> 1) * 8;
+    ldsm_x4(smem_u32(ah + aoff), af);
+    if constexpr (!BF16) ldsm_x4(smem_u32(al + aoff), afl);
+#pragma unroll
+    for (int np = 0; np < NTW / 2; ++np) {
+      uint32_t rh[4], rl[4];
+      const int boff = (16 * ks + lr + (li & 1) * 8) * BP + n0 + 16 * np + (li >> 1) * 8;
+      ldsm_x4_t(smem_u32(bh + boff), rh);
+      ldsm_x4_t(smem_u32(bl + boff), rl);
+      mma_bf16(acc[2 * np], af, rh[0], rh[1]);
+      mma_bf16(acc[2 * np], af, rl[0], rl[1]);
+      mma_bf16(acc[2 * np + 1], af, rh[2], rh[3]);
+      mma_bf16(acc[2 * np + 1], af, rl[2], rl[3]);
+      if constexpr (!BF16) {
+        mma_bf16(acc[2 * np], afl, rh[0], rh[1]);
+        mma_bf16(acc[2 * np + 1], afl, rh[2], rh[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int hi8 = 0; hi8 < 2; ++hi8) {
+    const int row = 16 * mt + g + 8 * hi8, tt = t0 + row;
+    if (tt >= a.n_sel) continue;
+    __nv_bfloat16 *o = a.out + ((size_t)tt * a.n_kv + h) * D + n0 + 2 * t;
+#pragma unroll
+    for (int n = 0; n < NTW; ++n)
+      *reinterpret_cast<uint32_t *>(o + 8 * n) = pack_bf16(acc[n][2 * hi8], acc[n][2 * hi8 + 1]);
   }
 }
 
@@ -446,17 +613,18 @@ cudaError_t factorize_r(XkArgs a, int iters, float *v_a, float *v_b, const float
   cudaError_t e;
   const int nt = a.F / kGramTile;
   const dim3 gg(nt * (nt + 1) / 2, a.n_kv, (a.S + a.tok_per_split - 1) / a.tok_per_split);
-  xkv_gram<<<gg, 128, 0, st>>>(a);
+  if ((e = ensure_smem_limit((const void *)xkv_gram, kGramSmem))) return e;
+  xkv_gram<<<gg, 128, kGramSmem, st>>>(a);
   count_launch();
   if ((e = cudaGetLastError())) return e;
   const int gv_smem = 2 * kGvK * (kRowsPerCta + R) * (int)sizeof(float);
-  const int chol_smem = (2 * R * (R + 1) + R) * (int)sizeof(double);
+  const int chol_smem = (3 * R * (R + 1) + R) * (int)sizeof(double);
   const int apply_smem = R * R * (int)sizeof(double) + kRowsPerCta * (R + 1) * (int)sizeof(float);
-  const int proj_smem = (a.F * R + 64 * 33) * (int)sizeof(float);
+  const int proj_smem = (2 * R * (a.F + 8) + 2 * kPjTok * kPjXP) * (int)sizeof(__nv_bfloat16);
   if ((e = ensure_smem_limit((const void *)xkv_gv<R>, gv_smem))) return e;
   if ((e = ensure_smem_limit((const void *)xkv_chol<R>, chol_smem))) return e;
   if ((e = ensure_smem_limit((const void *)xkv_apply<R>, apply_smem))) return e;
-  if ((e = ensure_smem_limit((const void *)xkv_project<R>, proj_smem))) return e;
+  if ((e = ensure_smem_limit((const void *)xkv_project_tc<R>, proj_smem))) return e;
   const dim3 rows(a.F / kRowsPerCta, a.n_kv);
   const float *cur = v0;
   for (int it = 0; it < iters; ++it) {
@@ -466,7 +634,7 @@ cudaError_t factorize_r(XkArgs a, int iters, float *v_a, float *v_b, const float
     xkv_gv<R><<<rows, 128, gv_smem, st>>>(a);
     count_launch();
     if ((e = cudaGetLastError())) return e;
-    xkv_chol<R><<<a.n_kv, 256, chol_smem, st>>>(a);
+    xkv_chol<R><<<a.n_kv, 512, chol_smem, st>>>(a);
     count_launch();
     if ((e = cudaGetLastError())) return e;
     xkv_apply<R><<<rows, 128, apply_smem, st>>>(a, it == iters - 1 ? 1 : 0);
@@ -474,24 +642,29 @@ cudaError_t factorize_r(XkArgs a, int iters, float *v_a, float *v_b, const float
     if ((e = cudaGetLastError())) return e;
     cur = nxt;
   }
-  a.v_final = cur;
-  xkv_project<R><<<dim3((a.S + 63) / 64, a.n_kv), 256, proj_smem, st>>>(a);
+  // about one CTA per SM over (token runs, heads)
+  const int n_tiles = (a.S + kPjTok - 1) / kPjTok;
+  const int ctas_per_head = std::max(1, std::min(n_tiles, (kNumSMs + a.n_kv - 1) / a.n_kv));
+  const int tiles_per_cta = (n_tiles + ctas_per_head - 1) / ctas_per_head;
+  xkv_project_tc<R><<<dim3((n_tiles + tiles_per_cta - 1) / tiles_per_cta, a.n_kv), 256, proj_smem, st>>>(a, tiles_per_cta);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int R, int D, bool BF16>
+cudaError_t rebuild_launch(const XrArgs &a, cudaStream_t st) {
+  constexpr int smem = RebuildLayout<R, D>::kBytes;
+  cudaError_t e = ensure_smem_limit((const void *)xkv_rebuild_tc<R, D, BF16>, smem);
+  if (e) return e;
+  xkv_rebuild_tc<R, D, BF16><<<dim3((a.n_sel + 63) / 64, a.n_kv), 256, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
 
 template <int R>
 cudaError_t rebuild_r(const XrArgs &a, bool bf16, cudaStream_t st) {
-  const dim3 grid((a.n_sel + 63) / 64, a.n_kv);
-  count_launch();
-  if (a.d == 128) {
-    if (bf16) xkv_rebuild<R, 128, true><<<grid, 256, 0, st>>>(a);
-    else xkv_rebuild<R, 128, false><<<grid, 256, 0, st>>>(a);
-  } else {
-    if (bf16) xkv_rebuild<R, 64, true><<<grid, 256, 0, st>>>(a);
-    else xkv_rebuild<R, 64, false><<<grid, 256, 0, st>>>(a);
-  }
-  return cudaGetLastError();
+  if (a.d == 128) return bf16 ? rebuild_launch<R, 128, true>(a, st) : rebuild_launch<R, 128, false>(a, st);
+  return bf16 ? rebuild_launch<R, 64, true>(a, st) : rebuild_launch<R, 64, false>(a, st);
 }
 
 }  // namespace
