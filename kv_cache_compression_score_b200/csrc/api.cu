@@ -104,6 +104,28 @@ kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int
     if (ctas <= target) break;
   }
   tpc = std::max(1, std::min(tpc, std::max(1, max_tiles)));
+  if (pl->tc) {
+    // the grid is (n_kv, chunks of the longest sequence, n_seqs); when it
+    // exceeds one CTA per SM the launch is not fused
+    const int64_t grid = (int64_t)n_kv * n_seqs * ((std::max(1, max_tiles) + tpc - 1) / tpc);
+    if (grid > kvc::kNumSMs) {
+      // the split launches (one CTA per SM, several waves): the chunk size
+      // that minimises waves x (tiles per chunk + a per-CTA setup cost of
+      // about 8 tiles), so that long sequences no longer set the makespan
+      auto cost = [&](int t) {
+        int64_t c = 0;
+        for (int b = 0; b < n_seqs; ++b) c += (int64_t)n_kv * ((tiles[b] + t - 1) / t);
+        return (c + kvc::kNumSMs - 1) / kvc::kNumSMs * (int64_t)(t + 8);
+      };
+      int best = tpc;
+      int64_t best_cost = cost(tpc);
+      for (int t = 4; t < max_tiles; ++t) {
+        const int64_t c = cost(t);
+        if (c < best_cost) { best_cost = c; best = t; }
+      }
+      tpc = best;
+    }
+  }
   pl->keys_per_chunk = tpc * pl->tile;
   pl->n_chunks = std::max(1, (pl->bt.max_len + pl->keys_per_chunk - 1) / pl->keys_per_chunk);
   // one cooperative launch when the whole grid is resident at once (one CTA per SM)
