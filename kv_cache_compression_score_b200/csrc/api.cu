@@ -134,7 +134,7 @@ kvc_status plan_score(kvc_dtype dt, int n_seqs, const int32_t *seqlens_host, int
   pl->off_sync = kErrWordBytes;
   pl->off_hist = round_up(pl->off_sync + units * kvc::tc_counters_per_unit() * sizeof(int), 256);
   pl->off_cnt = round_up(pl->off_hist + units * kvc::tc_hist_ints() * sizeof(int), 256);
-  pl->off_part = round_up(pl->off_cnt + units * pl->n_chunks * 2 * sizeof(int), 256);
+  pl->off_part = round_up(pl->off_cnt + units * pl->n_chunks * kvc::tc_count_ints() * sizeof(int), 256);
   const size_t part_bytes = (size_t)n_seqs * n_kv * pl->n_chunks * pl->R_pad * sizeof(float2);
   pl->off_raw = round_up(pl->off_part + part_bytes, 256);
   pl->bytes = pl->off_raw + round_up((size_t)n_kv * pl->bt.T * sizeof(float), 256);

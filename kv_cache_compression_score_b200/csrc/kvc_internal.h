@@ -46,6 +46,7 @@ int simt_keys_per_tile();
 int tc_keys_per_tile();
 int tc_counters_per_unit();   // fused launch: arrival counters per (sequence, KV head)
 int tc_hist_ints();           // fused selection: histogram ints per (sequence, KV head)
+int tc_count_ints();          // fused selection: count ints per (sequence, KV head, key chunk)
 int tc_select_max_keys(int d_h);  // fused selection: largest key chunk it keeps on chip
 
 cudaError_t pool_prefix(const float *raw, float *scores, const int32_t *cu_seqlens, int n_seqs, int n_kv,

@@ -107,9 +107,10 @@ struct TcParams {
 };
 
 // fused selection: counters and per-(sequence, head) radix histograms
-constexpr int kCtrPerUnit = 8;     // stats, raw, depart, radix levels 1-3, counts, spare
+constexpr int kCtrPerUnit = 8;     // stats, raw, depart, radix levels 1-3, two spare
 constexpr int kH1 = 4096, kH2 = 4096, kH3 = 256;
 constexpr int kHistInts = kH1 + kH2 + kH3;
+constexpr int kCntInts = 2 + kH3;  // per (sequence, head, chunk): keys above the 24-bit prefix, spare, level-3 bins
 // keys of one chunk held in shared memory: the K ring (kStages tiles of kBN x d_h bf16) as uint32
 
 // Shared-memory objects of one CTA.
@@ -565,12 +566,14 @@ KVC_DEVINL void find_bucket_from_top(const int *hist, int nbins, int need, int *
 //   adds its histogram of the candidates to a per-head histogram in the
 //   workspace, waits on a counter, and reads the bucket holding the k-th key.
 //   (A single log-scale bucket with a candidate exchange was tried: pooled
-//   scores crowd into few buckets, so it was slower.)  Then every CTA
-//   publishes its counts of keys > T and == T, and writes its kept positions
-//   at (keys > T in earlier chunks) + (equal keys taken in earlier chunks) +
-//   its own rank, which gives the ascending order and the lowest-position tie
-//   rule across chunks.  The CTA gathers the rows it placed; the CTA holding
-//   position P writes and gathers the window.
+//   scores crowd into few buckets, so it was slower.)  With its level-3
+//   histogram every CTA also publishes its own 256 level-3 bins and its count
+//   of keys above the 24-bit prefix; once T is known, the keys > T and == T
+//   of every earlier chunk follow from those records without another round.
+//   A CTA writes its kept positions at (keys > T in earlier chunks) + (equal
+//   keys taken in earlier chunks) + its own rank, which gives the ascending
+//   order and the lowest-position tie rule across chunks.  The CTA gathers the
+//   rows it placed; the CTA holding position P writes and gathers the window.
 template <int D>
 KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const TcWork &wk, int *ctr, int nc,
                                     const uint32_t *keys) {
@@ -584,7 +587,7 @@ KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const T
   int *scr = reinterpret_cast<int *>(sm.xch);        // scan scratch
   int *sh = reinterpret_cast<int *>(sm.sq);          // shared histogram (the window block is free)
   int *hist = p.hist + (size_t)(wk.b * p.n_kv + wk.h) * kHistInts;
-  int *cnt = p.cnt + (size_t)(wk.b * p.n_kv + wk.h) * p.n_chunks * 2;
+  int *cnt = p.cnt + (size_t)(wk.b * p.n_kv + wk.h) * p.n_chunks * kCntInts;
 
   uint32_t T = 0;
   int need = 0;                                     // keys equal to T to take over the head
@@ -592,20 +595,32 @@ KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const T
   if (!all && k_sel > 0) {
     uint32_t fixed = 0;                              // key bits fixed by the earlier levels
     need = k_sel;
+    int *above24 = scr + 96;                         // this chunk's keys above the 24-bit prefix (level 3)
     for (int lvl = 0; lvl < 3; ++lvl) {
       const int nbins = lvl < 2 ? 4096 : 256;
       const int shift = lvl == 0 ? 20 : (lvl == 1 ? 8 : 0);
       int *gh = hist + (lvl == 0 ? 0 : (lvl == 1 ? kH1 : kH1 + kH2));
       for (int b = tid; b < nbins; b += kThreadsTC) sh[b] = 0;
+      if (tid == 0) *above24 = 0;
       __syncthreads();
+      int my_above = 0;
       for (int i = tid; i < n_my; i += kThreadsTC) {
         const uint32_t kk = keys[i];
         const bool cand = lvl == 0 || (lvl == 1 ? (kk >> 20) == fixed : (kk >> 8) == fixed);
         if (cand) atomicAdd(&sh[(kk >> shift) & (nbins - 1)], 1);
+        if (lvl == 2) my_above += (kk >> 8) > fixed;
       }
+      if (lvl == 2 && my_above) atomicAdd(above24, my_above);
       __syncthreads();
       for (int b = tid; b < nbins; b += kThreadsTC)
         if (sh[b]) atomicAdd(&gh[b], sh[b]);
+      if (lvl == 2) {
+        // this chunk's level-3 record, read by the later chunks of the head
+        // after the level-3 counter (so no separate round for the counts)
+        int *rec = cnt + (size_t)wk.c * kCntInts;
+        for (int b = tid; b < kH3; b += kThreadsTC) rec[2 + b] = sh[b];
+        if (tid == 0) rec[0] = *above24;
+      }
       __syncthreads();
       if (tid == 0 && !arrive_and_wait(&ctr[3 + lvl], nc)) *sm.cta_err = 1;
       __syncthreads();
@@ -615,29 +630,20 @@ KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const T
       fixed = lvl == 0 ? (uint32_t)bin : (fixed << (lvl == 1 ? 12 : 8)) | (uint32_t)bin;
     }
     T = fixed;
-    // ---- counts of keys > T and == T per chunk, then the earlier chunks' sums
+    // ---- keys > T and == T in the earlier chunks, from their level-3
+    // records: keys above the 24-bit prefix plus the bins above / at T's bin
+    const int tb = (int)(T & 255u);
     int gt = 0, eq = 0;
-    for (int i = tid; i < n_my; i += kThreadsTC) {
-      gt += keys[i] > T;
-      eq += keys[i] == T;
+    for (int e = tid; e < wk.c * kCntInts; e += kThreadsTC) {
+      const int f = e % kCntInts;
+      if (f == 1) continue;
+      const int v = __ldcg(cnt + e);
+      if (f == 0) gt += v;
+      else if (f - 2 > tb) gt += v;
+      else if (f - 2 == tb) eq += v;
     }
-    int tot_gt, tot_eq;
-    block_exclusive_scan(gt, scr, &tot_gt);
-    block_exclusive_scan(eq, scr, &tot_eq);
-    if (tid == 0) {
-      cnt[2 * wk.c] = tot_gt;
-      cnt[2 * wk.c + 1] = tot_eq;
-      if (!arrive_and_wait(&ctr[6], nc)) *sm.cta_err = 1;
-    }
-    __syncthreads();
-    int2 c2 = make_int2(0, 0);
-    for (int cc = tid; cc < wk.c; cc += kThreadsTC) {
-      const int2 v = __ldcg(reinterpret_cast<const int2 *>(cnt) + cc);
-      c2.x += v.x;
-      c2.y += v.y;
-    }
-    block_exclusive_scan(c2.x, scr, &base_gt);
-    block_exclusive_scan(c2.y, scr, &base_eq);
+    block_exclusive_scan(gt, scr, &base_gt);
+    block_exclusive_scan(eq, scr, &base_eq);
   }
 
   // ---- this chunk's output offset and its share of the equal keys
@@ -863,6 +869,7 @@ cudaError_t launch_tc(const ScoreArgs &a, cudaStream_t st) {
 int tc_keys_per_tile() { return kBN; }
 int tc_counters_per_unit() { return kCtrPerUnit; }
 int tc_hist_ints() { return kHistInts; }
+int tc_count_ints() { return kCntInts; }
 int tc_select_max_keys(int d_h) { return kStages * kBN * d_h * 2 / 4; }
 
 cudaError_t score_window_tc(const ScoreArgs &a, cudaStream_t st) {
