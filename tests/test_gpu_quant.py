@@ -114,3 +114,42 @@ def test_decode_q8_llama8b_batch16():
     err = float(np.abs(got - ref).max())
     log_parity(dict(what="decode_q8", d_h=d, batch=nb, rows=nb * B, max_abs_err=err))
     assert err <= DECODE_ATOL["bf16"], err
+
+
+def test_gather_q8_exact_ties_and_tiny_scales():
+    """Quotients that land exactly on half-integers (round half to even),
+    scales below the smallest normal float, all-zero vectors and seeded rows:
+    codes and scales bit-identical to the oracle's float32 quantiser."""
+    n_kv, d = 2, 128
+    rows = []
+    halves = np.arange(d, dtype=np.float64) - 63.5                     # -63.5 .. 63.5: x / 1 = k + 0.5
+    r0 = halves.copy(); r0[0] = 127.0                                   # amax 127: scale exactly 1
+    r1 = halves / 2.0; r1[5] = -63.5                                    # amax 63.5: scale exactly 0.5
+    r2 = np.zeros(d); r2[0] = 2.0 ** -127; r2[1:9] = 2.0 ** -128; r2[9] = -(2.0 ** -128)   # subnormal scale, ties
+    r3 = np.zeros(d)                                                    # all zero: scale 0, codes 0
+    kr, vr = synth.keys_values(3500, 0, 4, n_kv, d, "f32")
+    for extra in (r0, r1, r2, r3):
+        rows.append(extra)
+    base = np.stack(rows)                                               # [4, d]
+    k64 = np.concatenate([np.repeat(base[:, None, :], n_kv, axis=1), kr.astype(np.float64)], axis=0)
+    v64 = np.concatenate([np.repeat(base[::-1, None, :], n_kv, axis=1), vr.astype(np.float64)], axis=0)
+    k_bits, v_bits = synth.round_to(k64, "bf16"), synth.round_to(v64, "bf16")
+    assert np.array_equal(synth.bf16_bits_to_f32(k_bits[:4]).astype(np.float64), k64[:4])   # exactly representable
+    N = k64.shape[0]
+    idx = np.broadcast_to(np.arange(N, dtype=np.int32), (n_kv, N)).copy()
+    cu = torch.tensor([0, N], dtype=torch.int32, device="cuda")
+    kq = torch.empty((N, n_kv, d), dtype=torch.int8, device="cuda")
+    vq = torch.empty_like(kq)
+    ks = torch.empty((n_kv, N), dtype=torch.float32, device="cuda")
+    vs = torch.empty_like(ks)
+    kvc.kvc_gather_kv_q8([N], cu, cu, N, torch.from_numpy(idx).cuda(), to_device(k_bits, "bf16"),
+                         to_device(v_bits, "bf16"), kq, vq, ks, vs)
+    torch.cuda.synchronize()
+    kq_o, vq_o, ks_o, vs_o = O.gather_kv_q8(k_bits, v_bits, idx.astype(np.int64), [0, N], N, "bf16")
+    assert np.array_equal(kq.cpu().numpy(), kq_o) and np.array_equal(vq.cpu().numpy(), vq_o)
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), ks_o.view(np.uint32))
+    assert np.array_equal(vs.cpu().numpy().view(np.uint32), vs_o.view(np.uint32))
+    # the tie rows really are ties: codes alternate by round-half-to-even
+    assert list(kq_o[0, 0, 1:4]) == [-62, -62, -60] and list(kq_o[0, 0, 63:67]) == [0, 0, 2, 2]
+    assert ks_o[0, 2] > 0 and ks_o[0, 2] < np.finfo(np.float32).tiny
+    assert kq_o[2, 0, 1] == 64 and kq_o[2, 0, 9] == -64
