@@ -245,16 +245,26 @@ KVC_DEVINL int ld_acquire(const int *p) {
   return v;
 }
 
-// One thread: announce this CTA on *ctr, then wait (bounded) until n CTAs did.
-KVC_DEVINL bool arrive_and_wait(int *ctr, int n) {
-  __threadfence();
-  atomicAdd(ctr, 1);
+// One thread: wait (bounded) until n CTAs have announced themselves on *ctr.
+KVC_DEVINL bool wait_count(const int *ctr, int n) {
   const uint64_t t0 = global_ns();
   while (ld_acquire(ctr) < n) {
     if (global_ns() - t0 > kWaitLimitNs) return false;
     __nanosleep(64);
   }
   return true;
+}
+
+// One thread: announce this CTA on *ctr (its earlier writes first).
+KVC_DEVINL void arrive(int *ctr) {
+  __threadfence();
+  atomicAdd(ctr, 1);
+}
+
+// One thread: announce this CTA on *ctr, then wait (bounded) until n CTAs did.
+KVC_DEVINL bool arrive_and_wait(int *ctr, int n) {
+  arrive(ctr);
+  return wait_count(ctr, n);
 }
 
 // One pass over the CTA's key chunk, all warp roles.
@@ -628,6 +638,18 @@ KVC_DEVINL void fused_select_gather(const TcParams &p, const TcSmem &sm, const T
       find_bucket_from_top(gh, nbins, need, scr, bin, above);
       need -= above;
       fixed = lvl == 0 ? (uint32_t)bin : (fixed << (lvl == 1 ? 12 : 8)) | (uint32_t)bin;
+      if (lvl == 0) {
+        // keys above the level-1 bucket are kept whatever T turns out to be:
+        // bring their V rows (not read by the scoring) into L2 for the gather
+        const size_t head_bytes = (size_t)D * 2;
+        for (int i = tid; i < n_my; i += kThreadsTC)
+          if ((keys[i] >> 20) > fixed) {
+            const uint8_t *row = p.v + ((size_t)(wk.t0 + j0 + i) * p.n_kv + wk.h) * head_bytes;
+#pragma unroll
+            for (size_t o = 0; o < head_bytes; o += 128)
+              asm volatile("prefetch.global.L2 [%0];" :: "l"(row + o));
+          }
+      }
     }
     T = fixed;
     // ---- keys > T and == T in the earlier chunks, from their level-3
@@ -754,24 +776,31 @@ score_fused_kernel(TcParams p) {
 
   tc_pass<D, true>(p, sm, wk, tmem_base, true);
 
-  // every chunk of this head has written its raw scores: pool the chunk
+  // pool the chunk once every chunk of this head has written its raw scores
   __syncthreads();
-  if (threadIdx.x == 0 && !arrive_and_wait(&ctr[1], nc)) *sm.cta_err = 1;
-  __syncthreads();
+  if (threadIdx.x == 0) arrive(&ctr[1]);
   {
     const float *src = p.raw + (size_t)wk.h * p.T_total + wk.t0;
     float *dst = p.scores + (size_t)wk.h * p.T_total + wk.t0;
     uint32_t *keys = reinterpret_cast<uint32_t *>(sm.sk);   // the K ring is no longer needed
     const int r = p.pool_r;
     // stage the chunk's raw scores and the halo in the (free) window-block
-    // area with coalesced loads; neighbours outside the prefix read as -inf
+    // area with coalesced loads; neighbours outside the prefix read as -inf.
+    // The chunk's own scores are staged while the other chunks finish; the
+    // halo after the counter.
     float *stage = reinterpret_cast<float *>(sm.sq);
-    const int s_lo = wk.key_begin - r, s_n = min(wk.key_end, wk.P) + r - s_lo;
+    const int own_end = min(wk.key_end, wk.P);
+    const int s_lo = wk.key_begin - r, s_n = own_end + r - s_lo;
     const bool staged = s_n <= TcLayout<D>::kQBytes / 4;
-    if (staged) {
-      for (int e = threadIdx.x; e < s_n; e += kThreadsTC) {
-        const int j = s_lo + e;
-        stage[e] = (j >= 0 && j < wk.P) ? __ldcg(src + j) : kNegInf;
+    if (staged)
+      for (int j = wk.key_begin + threadIdx.x; j < own_end; j += kThreadsTC) stage[j - s_lo] = __ldcg(src + j);
+    __syncthreads();
+    if (threadIdx.x == 0 && !wait_count(&ctr[1], nc)) *sm.cta_err = 1;
+    __syncthreads();
+    if (staged && own_end > wk.key_begin) {          // (a chunk inside the window pools nothing)
+      for (int e = threadIdx.x; e < 2 * r; e += kThreadsTC) {
+        const int j = e < r ? s_lo + e : own_end + (e - r);
+        stage[j - s_lo] = (j >= 0 && j < wk.P) ? __ldcg(src + j) : kNegInf;
       }
       __syncthreads();
     }
