@@ -26,9 +26,9 @@ import pytest
 import torch
 
 from kv_cache_compression_score_b200 import kvc, synth
-from kv_cache_compression_score_b200.runner import to_device
+from kv_cache_compression_score_b200.runner import Decoder, from_device, to_device
 from oracle import kvc_oracle as O
-from parity_helpers import log_parity
+from parity_helpers import DECODE_ATOL, log_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -132,3 +132,48 @@ def test_xkv_out_of_range_rows_are_zero():
         assert np.all(o[t, h] == 0.0)
     for h, t in [(0, 0), (0, 3), (1, 1), (1, 2)]:
         assert np.any(o[t, h] != 0.0)
+
+
+def test_xkv_rebuilt_rows_feed_decode():
+    """Rows rebuilt by kvc_xkv_reconstruct are a compact cache in the decode
+    layout: decode over them matches the oracle's decode over the oracle's
+    bf16-rounded rebuilt rows (the same rows up to the bound above)."""
+    S, n_kv, d, W, r, n_sel, n_h = 4096, 8, 128, 4, 64, 512, 32
+    keys = synth.cross_layer_keys(4300, S, n_kv, d, W, r)
+    vals = synth.cross_layer_keys(4301, S, n_kv, d, W, r)
+    _, kb, kt = _factorize(keys, r, 8, torch.bfloat16, 4302)
+    _, vb, vt = _factorize(vals, r, 8, torch.bfloat16, 4303)
+    idx = synth.index_lists(4304, [S], n_kv, n_sel)
+    idx_dev = torch.from_numpy(idx).cuda()
+    layer = 2
+    kc = torch.empty((n_sel, n_kv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.empty_like(kc)
+    kvc.kvc_xkv_reconstruct(W, layer, kb, kt, idx_dev, kc)
+    kvc.kvc_xkv_reconstruct(W, layer, vb, vt, idx_dev, vc)
+    q = synth.decode_queries(4305, 1, n_h, d, "bf16")
+    dec = Decoder(1, n_h, n_kv, d, n_sel)
+    off = torch.zeros(1, dtype=torch.int64, device="cuda")
+    ln = torch.full((1,), n_sel, dtype=torch.int32, device="cuda")
+    dec.run(to_device(q, "bf16"), kc, vc, off, ln)
+    torch.cuda.synchronize()
+    got = dec.out.cpu().numpy().astype(np.float64)
+    # decode over the GPU's rebuilt rows, in the oracle
+    ref_gpu_rows = O.gqa_decode(q, from_device(kc), from_device(vc), [0], [n_sel], n_kv, "bf16")
+    assert np.abs(got - ref_gpu_rows).max() <= DECODE_ATOL["bf16"]
+    # and against decode over the oracle's own rebuilt rows (bf16): to first
+    # order, perturbing V by dV and the logits by dz moves each output by at
+    # most |dV|_inf + 2 |dz|_inf |V|_inf (the softmax weights move by at most
+    # 2 p_t |dz|_inf and sum to 1); a factor 1.5 covers the second order
+    A_k, Vt_k = O.xkv_factorize(keys, r, "bf16")
+    A_v, Vt_v = O.xkv_factorize(vals, r, "bf16")
+    rk = synth.round_to(O.xkv_reconstruct(A_k, Vt_k, layer, d, idx), "bf16")
+    rv = synth.round_to(O.xkv_reconstruct(A_v, Vt_v, layer, d, idx), "bf16")
+    ref = O.gqa_decode(q, rk, rv, [0], [n_sel], n_kv, "bf16")
+    kg, vg = O.to_f64(from_device(kc), "bf16"), O.to_f64(from_device(vc), "bf16")
+    ko, vo = O.to_f64(rk, "bf16"), O.to_f64(rv, "bf16")
+    qf = O.to_f64(q, "bf16")[0].reshape(n_kv, n_h // n_kv, d)
+    dz = np.abs(np.einsum("hgd,thd->thg", qf, kg - ko)).max() / np.sqrt(d)
+    tol = 1.5 * (np.abs(vg - vo).max() + 2.0 * dz * np.abs(vo).max()) + DECODE_ATOL["bf16"]
+    err = float(np.abs(got - ref).max())
+    log_parity({"test": "xkv_decode", "S": S, "n_sel": n_sel, "max_abs_err": err, "tol": float(tol)})
+    assert err <= tol, (err, tol)
