@@ -2,7 +2,9 @@
  * kvc.h -- C ABI of libkvc, the B200 (sm_100a) hot path of observation-window
  * KV-cache compression: window saliency scoring, budgeted per-KV-head top-k,
  * compact KV gather, GQA decode attention over the compact cache, and
- * FastKV-style token-selective propagation (TSP).
+ * FastKV-style token-selective propagation (TSP); with FreeKV's decode-time
+ * correction, per-layer budgets, an int8 compact cache, and xKV's cross-layer
+ * factorisation with selective reconstruction.
  *
  * Sources of the method (web pages; the library implements their outline and
  * states its readings of the points they leave open):
@@ -11,14 +13,20 @@
  *     "Quand la reutilisation est-elle exacte ?" (causal offset of appended
  *     rows; original positions kept after eviction), section "Compresser un
  *     cache existant" (SnapKV observation-window scoring; sliding windows keep
- *     a recent region).
+ *     a recent region; PyramidKV's per-layer budgets; a cache stored at lower
+ *     precision).
  *   - "FastKV: Decoupling of Context Reduction and KV Cache Compression for
  *     Prefill-Decoding Acceleration" (gist.science 2502.01068): section 2.A
  *     (token-selective propagation from window-attention saliency), section
  *     2.B (TSP rate independent of the KV retention rate).
  *   - "FreeKV: Boosting KV Cache Retrieval for Efficient LLM Inference"
- *     (gist.science 2505.13109), technical summary section 2.B: NHD layout on
- *     the GPU, which every cache tensor here uses.
+ *     (gist.science 2505.13109), technical summary section 2.A (speculative
+ *     retrieval with fine-grained correction) and section 2.B (NHD layout on
+ *     the GPU, which every cache tensor here uses).
+ *   - "xKV - Compression de Cache KV Inter-couche par Extraction de Vecteurs
+ *     Singuliers Alignes" (gist.science 2503.18893), technical summary
+ *     sections 2.2 (cross-layer factorisation) and 2.3 (selective
+ *     reconstruction).
  *
  * Conventions shared by every entry point
  *   - All calls are asynchronous on the caller's stream (a cudaStream_t passed
