@@ -241,6 +241,7 @@ gqa_decode_mma(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     // bf16 caches: dims 16ks + 2t (+1) and 16ks + 8 + 2t (+1); int8 caches:
     // dims 16ks + 4t .. 16ks + 4t + 3 (the order of the widened K codes).
     uint32_t qf[NKS][2];
+    float cz0 = p.c, cz1 = p.c;  // logit factors of heads 2t, 2t+1 (int8: divided by the query's power-of-two scale)
     float m[2], l[2], acc[NKS][4];
     int cur_b = -1, cur_h = -1;
     int64_t seg_u0 = 0;          // first flattened row of the current unit
@@ -248,19 +249,43 @@ gqa_decode_mma(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
 
     auto reset_unit = [&]() {
       const __nv_bfloat16 *qb = p.q + ((size_t)wk.b * p.n_h + (size_t)wk.h * G + g) * D;
+      if constexpr (Q8) {
+        // int8 caches: the query in f16, head g scaled by a power of two so
+        // that its largest element lies in [2^13, 2^14): every element within
+        // 2^27 of that largest converts exactly (bf16 carries 8 significant
+        // bits); the logit factor divides the scale out again
+        float qv[NKS][4];
+        float mx = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < NKS; ++ks) {
-        if (g < G) {
-          if constexpr (Q8) {
-            const uint2 q2 = __ldg(reinterpret_cast<const uint2 *>(qb + 16 * ks + 4 * t));
-            qf[ks][0] = q2.x;
-            qf[ks][1] = q2.y;
-          } else {
+        for (int ks = 0; ks < NKS; ++ks) {
+          uint2 q2 = make_uint2(0u, 0u);
+          if (g < G) q2 = __ldg(reinterpret_cast<const uint2 *>(qb + 16 * ks + 4 * t));
+          qv[ks][0] = bf16_lo(q2.x); qv[ks][1] = bf16_hi(q2.x); qv[ks][2] = bf16_lo(q2.y); qv[ks][3] = bf16_hi(q2.y);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qv[ks][e]));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        int ex = 0;
+        if (mx > 0.f) frexpf(mx, &ex);
+        const float qs = mx > 0.f ? ldexpf(1.f, 14 - ex) : 1.f;
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+          qf[ks][0] = pack_f16(qv[ks][0] * qs, qv[ks][1] * qs);
+          qf[ks][1] = pack_f16(qv[ks][2] * qs, qv[ks][3] * qs);
+        }
+        const float qinv = 1.f / qs;     // a power of two: exact
+        cz0 = p.c * __shfl_sync(0xffffffffu, qinv, 8 * t);       // head 2t lives in lanes 8t .. 8t + 3
+        cz1 = p.c * __shfl_sync(0xffffffffu, qinv, 8 * t + 4);   // head 2t + 1 in lanes 8t + 4 .. 8t + 7
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+          if (g < G) {
             qf[ks][0] = __ldg(reinterpret_cast<const uint32_t *>(qb + 16 * ks + 2 * t));
             qf[ks][1] = __ldg(reinterpret_cast<const uint32_t *>(qb + 16 * ks + 8 + 2 * t));
+          } else {
+            qf[ks][0] = qf[ks][1] = 0u;
           }
-        } else {
-          qf[ks][0] = qf[ks][1] = 0u;
         }
       }
       m[0] = m[1] = kNegInf;
@@ -366,25 +391,24 @@ gqa_decode_mma(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
                 // rows g, g+8 of the group; dims 16ks + 4t .. +3 of each
                 const uint32_t w0 = *reinterpret_cast<const uint32_t *>(stg_k + swz<L::kBoxB, kTR>(16 * gr + g, ks) + 4 * t);
                 const uint32_t w1 = *reinterpret_cast<const uint32_t *>(stg_k + swz<L::kBoxB, kTR>(16 * gr + g + 8, ks) + 4 * t);
-                a[0] = i8pair_bf16(w0, 0, w0, 8);
-                a[2] = i8pair_bf16(w0, 16, w0, 24);
-                a[1] = i8pair_bf16(w1, 0, w1, 8);
-                a[3] = i8pair_bf16(w1, 16, w1, 24);
+                i8x4_f16(w0, a[0], a[2]);
+                i8x4_f16(w1, a[1], a[3]);
+                mma_f16(sc[gr], a, qf[ks][0], qf[ks][1]);
               } else {
                 // matrices: (rows 0-7, dims 0-7), (rows 8-15, dims 0-7), (rows 0-7, dims 8-15), (rows 8-15, dims 8-15)
                 ldsm_x4(k_base + swz<128, kTR>(16 * gr + lr + (li & 1) * 8, 2 * ks + (li >> 1)), a);
+                mma_bf16(sc[gr], a, qf[ks][0], qf[ks][1]);
               }
-              mma_bf16(sc[gr], a, qf[ks][0], qf[ks][1]);
             }
           }
           // logits in log2 units: (row g, heads 2t, 2t+1), (row g+8, same heads)
           float z[2][4];
 #pragma unroll
           for (int gr = 0; gr < 2; ++gr) {
-            z[gr][0] = vr[gr][0] ? sc[gr][0] * p.c * ksc[gr][0] : kNegInf;
-            z[gr][1] = vr[gr][0] ? sc[gr][1] * p.c * ksc[gr][0] : kNegInf;
-            z[gr][2] = vr[gr][1] ? sc[gr][2] * p.c * ksc[gr][1] : kNegInf;
-            z[gr][3] = vr[gr][1] ? sc[gr][3] * p.c * ksc[gr][1] : kNegInf;
+            z[gr][0] = vr[gr][0] ? sc[gr][0] * cz0 * ksc[gr][0] : kNegInf;
+            z[gr][1] = vr[gr][0] ? sc[gr][1] * cz1 * ksc[gr][0] : kNegInf;
+            z[gr][2] = vr[gr][1] ? sc[gr][2] * cz0 * ksc[gr][1] : kNegInf;
+            z[gr][3] = vr[gr][1] ? sc[gr][3] * cz1 * ksc[gr][1] : kNegInf;
           }
           float tmax0 = fmaxf(fmaxf(z[0][0], z[0][2]), fmaxf(z[1][0], z[1][2]));
           float tmax1 = fmaxf(fmaxf(z[0][1], z[0][3]), fmaxf(z[1][1], z[1][3]));
