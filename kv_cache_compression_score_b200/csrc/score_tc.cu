@@ -762,17 +762,24 @@ score_fused_kernel(TcParams p) {
 
   tc_pass<D, false>(p, sm, wk, tmem_base, false);
 
-  // every chunk of this head has published its stats partial
+  // announce this chunk's stats partial; the loaders and the MMA thread start
+  // the score pass on the resident tiles at once (its products do not depend
+  // on the offsets), while the epilogue waits until every chunk of this head
+  // has published its partial and merges the offsets
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    if (!arrive_and_wait(&ctr[0], nc)) *sm.cta_err = 1;
+    arrive(&ctr[0]);
     init_pass_barriers(sm, true);
     fence_mbar_init();
   }
   __syncthreads();
   tc_fence_after();
-  if (warp_id() >= kEpiWarp0) merge_offsets(p, sm, wk);
+  if (warp_id() >= kEpiWarp0) {
+    if (threadIdx.x == kEpiWarp0 * 32 && !wait_count(&ctr[0], nc)) *sm.cta_err = 1;
+    asm volatile("bar.sync 1, %0;" :: "n"(kEpiWarps * 32) : "memory");
+    merge_offsets(p, sm, wk);
+  }
 
   tc_pass<D, true>(p, sm, wk, tmem_base, true);
 
