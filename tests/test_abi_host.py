@@ -203,3 +203,60 @@ def test_compress_window_rejects_before_launch(L):
     assert call(w=101) == INVALID                        # the second sequence is shorter than the window
     assert call(ws_bytes=64) == WORKSPACE
     assert call(dt=5) == UNSUPPORTED
+
+
+def test_int8_cache_calls_reject_before_launch(L):
+    """kvc_gather_kv_q8 and kvc_gqa_decode_attn_q8 validate every argument
+    before anything is launched (each call below has exactly one bad one)."""
+    sl = np.array([100, 40], np.int32)
+    slp = sl.ctypes.data_as(ctypes.c_void_p)
+
+    def gq(n_seqs=2, cu=P16, n_kv=8, d_h=128, budget=64, k_q=P16, pitch=104):
+        return L.kvc_gather_kv_q8(n_seqs, slp, cu, P16, n_kv, d_h, budget, P16, P16, P16, k_q, P16, P16, P16, pitch,
+                                  None)
+
+    assert gq(n_seqs=0) == INVALID
+    assert gq(n_kv=0) == INVALID
+    assert gq(d_h=96) == UNSUPPORTED
+    assert gq(budget=-1) == INVALID
+    assert gq(cu=None) == INVALID
+    assert gq(k_q=P8) == INVALID
+    assert gq(pitch=103) == INVALID and b"scale_pitch" in L.kvc_last_error()   # 64 + 40 compact rows
+    assert gq(budget=0) == 0                               # no compact rows: nothing to do, nothing launched
+
+    def dq(batch=2, n_h=32, d_h=128, q=P16, kv_len=P16, pitch=200, rows=200, ws_bytes=1 << 30):
+        return L.kvc_gqa_decode_attn_q8(batch, n_h, 8, d_h, 0.0, q, P16, P16, P16, P16, pitch, rows, P16, kv_len, 100,
+                                        P16, P16, ws_bytes, None)
+
+    assert dq(batch=0) == INVALID
+    assert dq(n_h=24) == UNSUPPORTED                       # GQA group 3
+    assert dq(d_h=80) == UNSUPPORTED
+    assert dq(q=P8) == INVALID
+    assert dq(kv_len=None) == INVALID
+    assert dq(rows=0) == INVALID
+    assert dq(pitch=199) == INVALID
+    assert dq(ws_bytes=8) == WORKSPACE
+
+
+def test_freekv_step_rejects_before_launch(L):
+    """kvc_freekv_step and its workspace query validate before any launch."""
+    sl = np.array([300, 100], np.int32)
+    slp = sl.ctypes.data_as(ctypes.c_void_p)
+    ws_ok = L.kvc_freekv_workspace_size(2, slp, 32, 8, 128, 32, 64)
+    assert ws_ok > 0
+    assert L.kvc_freekv_workspace_size(2, slp, 32, 8, 128, 32, 31) == 0     # budget below the window
+    assert L.kvc_freekv_workspace_size(2, slp, 32, 8, 128, 101, 128) == 0   # a sequence shorter than w
+    assert L.kvc_freekv_workspace_size(2, slp, 24, 8, 128, 32, 64) == 0     # GQA group 3
+    assert L.kvc_freekv_workspace_size(2, slp, 32, 8, 96, 32, 64) == 0      # d_h
+
+    def fk(pool_k=7, budget=64, cu_budget=P16, q_prev=P16, out=P16, ws_bytes=ws_ok):
+        return L.kvc_freekv_step(2, slp, P16, cu_budget, 32, 8, 128, 32, pool_k, budget, 0.9, 0.0, P16, q_prev,
+                                 P16, P16, P16, P16, P16, P16, out, P16, ws_bytes, None)
+
+    assert fk(pool_k=6) == INVALID
+    assert fk(pool_k=33) == INVALID
+    assert fk(budget=31) == INVALID and b"window" in L.kvc_last_error()
+    assert fk(cu_budget=None) == INVALID
+    assert fk(q_prev=P8) == INVALID
+    assert fk(out=None) == INVALID
+    assert fk(ws_bytes=ws_ok - 1) == WORKSPACE
