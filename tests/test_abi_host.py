@@ -260,3 +260,18 @@ def test_freekv_step_rejects_before_launch(L):
     assert fk(q_prev=P8) == INVALID
     assert fk(out=None) == INVALID
     assert fk(ws_bytes=ws_ok - 1) == WORKSPACE
+
+
+def test_tsp_static_rejects_before_launch(L):
+    """The no-allocation TSP entry point checks its size limit and every
+    argument before it resolves its scratch or launches anything."""
+    def ts(S=1000, w=32, pool_k=7, k_tsp=100, D=4096, hidden=P16, dt=kvc.KVC_BF16):
+        return L.kvc_tsp_select_gather_static(dt, S, 8, w, pool_k, k_tsp, P16, hidden, D, P16, P16, None)
+
+    assert ts(S=262144 + 33) == UNSUPPORTED and b"workspace" in L.kvc_last_error()   # S - w = 262,145
+    assert ts(dt=7) == UNSUPPORTED
+    assert ts(w=1001) == INVALID
+    assert ts(pool_k=8) == INVALID
+    assert ts(k_tsp=969) == INVALID                        # beyond the prefix S - w = 968
+    assert ts(D=4) == UNSUPPORTED                          # 8-byte rows
+    assert ts(hidden=P8) == INVALID
