@@ -35,12 +35,13 @@
 //
 // When the whole grid fits on the GPU at once (one CTA per SM), both passes
 // and the max-pool run in ONE cooperative launch: a CTA publishes its stats
-// partial, waits on a per-(sequence, head) arrival counter for the other key
-// chunks of its head, then runs the score pass over its own chunk in reverse
-// tile order -- the last kStages tiles of the stats pass are still in its
-// shared-memory ring and are not loaded again, the rest mostly come from L2 --
-// and after a second counter pools its chunk (halo from the neighbours' raw
-// scores).  This saves a launch, the window-block staging, the tensor-memory
+// partial and runs the score pass over its own chunk in reverse tile order --
+// the last kStages tiles of the stats pass are still in its shared-memory
+// ring and are not loaded again, the rest mostly come from L2.  Its loaders
+// and MMA thread start at once (the products need no offsets) while its
+// epilogue waits on a per-(sequence, head) arrival counter for the other key
+// chunks of its head and merges the offsets.  After a second counter it pools
+// its chunk (halo from the neighbours' raw scores).  This saves a launch, the window-block staging, the tensor-memory
 // allocation and the separate pool kernel, and a third of the second K pass.
 // Otherwise the two passes are separate launches and the pool kernel follows.
 // Every wait is bounded; a wait that gives up sets the device error word and
